@@ -1,0 +1,227 @@
+// The C ABI of liblvq: argument validation, layouts, and kernel launches.
+#include <math.h>
+#include <string.h>
+
+#include "lvq_common.cuh"
+
+using namespace lvq;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// LoopVQ shape rules ("LoopVQ summary", "how it differs": Tc divides T and G,
+// one code covers c = G/Tc channels of each step; "premises and limits": 8-bit
+// codes, K = 256, 8-token pages), then this build's kernel set.
+lvq_status check_cfg(const lvq_config* c) {
+  if (!c) return LVQ_EINVAL;
+  if (c->n_layers < 1 || c->n_kv_heads < 1 || c->n_q_heads < 1 || c->head_dim < 2 || c->T < 1 ||
+      c->Tc < 1 || c->G < 1 || c->n_sink < 0 || c->n_recent < 0 || c->max_batch < 1 ||
+      c->max_ctx < 1 || c->max_splits < 1 || !(c->rope_base > 0.f) || !isfinite(c->rope_base))
+    return LVQ_EINVAL;
+  if (c->T % c->Tc || c->G % c->Tc || c->n_q_heads % c->n_kv_heads || c->head_dim % 2)
+    return LVQ_EINVAL;
+  const int cc = c->G / c->Tc;
+  if (c->head_dim % cc || (c->head_dim / cc) % 2) return LVQ_EINVAL;
+  if (c->K != kEntries || c->page_tokens != kPage) return LVQ_EUNSUPPORTED;
+  if (!decode_supported(c->head_dim, cc) || !encode_supported(c->G, cc)) return LVQ_EUNSUPPORTED;
+  if (c->max_splits > 1024 || c->max_ctx > (1 << 28)) return LVQ_EUNSUPPORTED;
+  return LVQ_OK;
+}
+
+Geo make_geo(const lvq_config* c) {
+  Geo g;
+  g.L = c->n_layers; g.H = c->n_kv_heads; g.Hq = c->n_q_heads; g.d = c->head_dim;
+  g.T = c->T; g.Tc = c->Tc; g.G = c->G; g.c = c->G / c->Tc; g.ng = g.d / g.c; g.nblk = g.T / g.Tc;
+  g.S = c->n_sink; g.W = c->n_recent; g.R = c->n_recent + kPage;
+  const int max_coded = c->max_ctx > c->n_sink ? c->max_ctx - c->n_sink : 0;
+  g.P = max_coded > 0 ? (max_coded + kPage - 1) / kPage : 1;
+  g.B = c->max_batch; g.max_ctx = c->max_ctx; g.max_splits = c->max_splits;
+  g.RC = (c->max_ctx + kPage - 1) / kPage + 16;
+  g.page_bytes = 2 * g.ng * kPage;
+  return g;
+}
+
+void fill_layout(const Geo& g, lvq_layout* o) {
+  memset(o, 0, sizeof(*o));
+  o->c = g.c; o->n_groups = g.ng; o->n_blocks = g.nblk; o->ring_tokens = g.R; o->max_pages = g.P;
+  o->page_bytes = g.page_bytes; o->rope_coarse = g.RC;
+  const int64_t idims[8] = {g.L, g.nblk, g.B, g.H, g.P, 2, g.ng, kPage};
+  int64_t st = 1;
+  for (int i = 7; i >= 0; --i) { o->idx_strides[i] = st; st *= idims[i]; }
+  o->idx_bytes = (size_t)st;
+  const int64_t cdims[7] = {g.L, 2, g.nblk, g.H, g.ng, kEntries, g.G};
+  st = 1;
+  for (int i = 6; i >= 0; --i) { o->cb_strides[i] = st; st *= cdims[i]; }
+  o->cb_bytes = (size_t)st * 2;
+  const int64_t pdims[8] = {g.L, 2, g.nblk, g.H, g.Tc, kEntries, g.ng, g.c};
+  st = 1;
+  for (int i = 7; i >= 0; --i) { o->cbp_strides[i] = st; st *= pdims[i]; }
+  o->cbp_bytes = (size_t)st * 2;
+  o->cb_norm_bytes = (size_t)g.L * 2 * g.nblk * g.H * g.ng * kEntries * 4;
+  const int64_t sdims[7] = {g.L, 2, g.T, g.B, g.H, g.S, g.d};
+  st = 1;
+  for (int i = 6; i >= 0; --i) { o->sink_strides[i] = st; st *= sdims[i]; }
+  o->sink_bytes = (size_t)st * 2;
+  const int64_t rdims[7] = {g.L, 2, g.T, g.B, g.H, g.R, g.d};
+  st = 1;
+  for (int i = 6; i >= 0; --i) { o->ring_strides[i] = st; st *= rdims[i]; }
+  o->ring_bytes = (size_t)st * 2;
+  o->rope_bytes = (size_t)(g.RC + kPage) * (g.d / 2) * 2 * 4;
+  o->workspace_bytes = (size_t)g.B * g.Hq * (g.max_splits + 1) * (g.d + 2) * 4;
+}
+
+// Re-derives the layout and checks the caller's copy matches it.
+lvq_status check_all(const lvq_config* cfg, const lvq_layout* lay, Geo* g) {
+  lvq_status s = check_cfg(cfg);
+  if (s != LVQ_OK) return s;
+  if (!lay) return LVQ_EINVAL;
+  *g = make_geo(cfg);
+  lvq_layout ref;
+  fill_layout(*g, &ref);
+  if (memcmp(&ref, lay, sizeof(ref)) != 0) return LVQ_EINVAL;
+  return LVQ_OK;
+}
+
+// The library runs on sm_100 devices only.
+lvq_status check_device() {
+  static int ok[kMaxDevices] = {};   // 0 unknown, 1 good, -1 bad
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return LVQ_EDEVICE;
+  if (dev < kMaxDevices && ok[dev] == 1) return LVQ_OK;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return LVQ_EDEVICE;
+  const bool good = major == 10;
+  if (dev < kMaxDevices) ok[dev] = good ? 1 : -1;
+  return good ? LVQ_OK : LVQ_EDEVICE;
+}
+
+lvq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LVQ_OK : LVQ_ECUDA; }
+
+}  // namespace
+
+extern "C" {
+
+lvq_status lvq_cache_layout(const lvq_config* cfg, lvq_layout* out) {
+  if (!out) return LVQ_EINVAL;
+  lvq_status s = check_cfg(cfg);
+  if (s != LVQ_OK) return s;
+  fill_layout(make_geo(cfg), out);
+  return LVQ_OK;
+}
+
+const char* lvq_status_string(lvq_status s) {
+  switch (s) {
+    case LVQ_OK: return "ok";
+    case LVQ_EINVAL: return "invalid argument";
+    case LVQ_EUNSUPPORTED: return "shape not supported by this build";
+    case LVQ_ECAPACITY: return "request exceeds the cache layout's capacity";
+    case LVQ_ECUDA: return "CUDA call or kernel launch failed";
+    case LVQ_ETIMEOUT: return "bounded device-side wait expired";
+    case LVQ_EDEVICE: return "no usable sm_100 device";
+  }
+  return "unknown status";
+}
+
+lvq_status lvq_pack_codebooks(const lvq_config* cfg, const lvq_layout* lay, const void* cb, void* cbp,
+                              float* cb_norm, void* stream) {
+  Geo g;
+  lvq_status s = check_all(cfg, lay, &g);
+  if (s != LVQ_OK) return s;
+  if (!cb || !cbp || !aligned16(cb) || !aligned16(cbp) || (cb_norm && !aligned16(cb_norm)))
+    return LVQ_EINVAL;
+  if ((s = check_device()) != LVQ_OK) return s;
+  return cuda_status(launch_pack(g, static_cast<const __nv_bfloat16*>(cb), static_cast<__nv_bfloat16*>(cbp),
+                                 cb_norm, static_cast<cudaStream_t>(stream)));
+}
+
+lvq_status lvq_rope_table(const lvq_config* cfg, const lvq_layout* lay, float* rope, void* stream) {
+  Geo g;
+  lvq_status s = check_all(cfg, lay, &g);
+  if (s != LVQ_OK) return s;
+  if (!rope || !aligned16(rope)) return LVQ_EINVAL;
+  if ((s = check_device()) != LVQ_OK) return s;
+  return cuda_status(launch_rope_table(g, cfg->rope_base, rope, static_cast<cudaStream_t>(stream)));
+}
+
+lvq_status lvq_encode_prefill(const lvq_config* cfg, const lvq_layout* lay, int32_t layer, int32_t req,
+                              const void* kv, int64_t kv_tok_stride, int32_t kv_tokens, int32_t tok_begin,
+                              int32_t n_tok, int32_t coded_offset, const void* cb, uint8_t* idx,
+                              int32_t* dev_status, void* stream) {
+  Geo g;
+  lvq_status s = check_all(cfg, lay, &g);
+  if (s != LVQ_OK) return s;
+  if (layer < 0 || layer >= g.L || req < 0 || req >= g.B || n_tok < 0 || tok_begin < 0 ||
+      kv_tokens < 0 || (int64_t)tok_begin + n_tok > kv_tokens || coded_offset < 0 ||
+      (int64_t)coded_offset + n_tok > (int64_t)g.P * kPage || kv_tok_stride < (int64_t)g.H * g.d)
+    return LVQ_EINVAL;
+  if (n_tok > 0 && (!kv || !cb || !idx || !aligned16(kv) || !aligned16(cb) || !aligned16(idx)))
+    return LVQ_EINVAL;
+  if ((s = check_device()) != LVQ_OK) return s;
+  return cuda_status(launch_encode_prefill(g, layer, req, static_cast<const __nv_bfloat16*>(kv), kv_tok_stride,
+                                           kv_tokens, tok_begin, n_tok, coded_offset,
+                                           static_cast<const __nv_bfloat16*>(cb), idx, dev_status,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+lvq_status lvq_encode_page(const lvq_config* cfg, const lvq_layout* lay, int32_t batch, const int32_t* ctx_len,
+                           int32_t* coded_len, const void* ring, const void* cb, uint8_t* idx,
+                           int32_t* dev_status, void* stream) {
+  Geo g;
+  lvq_status s = check_all(cfg, lay, &g);
+  if (s != LVQ_OK) return s;
+  if (batch < 0 || batch > g.B) return LVQ_EINVAL;
+  if (batch > 0 && (!ctx_len || !coded_len || !ring || !cb || !idx || !aligned16(ring) || !aligned16(cb) ||
+                    !aligned16(idx)))
+    return LVQ_EINVAL;
+  if ((s = check_device()) != LVQ_OK) return s;
+  return cuda_status(launch_encode_page(g, batch, ctx_len, coded_len, static_cast<const __nv_bfloat16*>(ring),
+                                        static_cast<const __nv_bfloat16*>(cb), idx, dev_status,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+lvq_status lvq_decode_attention(const lvq_config* cfg, const lvq_layout* lay, int32_t layer, int32_t step,
+                                int32_t batch, const void* q, const int32_t* ctx_len,
+                                const int32_t* coded_len, const void* sink, const void* ring,
+                                const uint8_t* idx, const void* cbp, const float* rope, int32_t num_splits,
+                                float* workspace, float* out, float* lse, float* split_lse,
+                                int32_t* dev_status, void* stream) {
+  Geo g;
+  lvq_status s = check_all(cfg, lay, &g);
+  if (s != LVQ_OK) return s;
+  if (layer < 0 || layer >= g.L || step < 0 || step >= g.T || batch < 0 || batch > g.B || num_splits < 1 ||
+      num_splits > g.max_splits)
+    return LVQ_EINVAL;
+  if (batch > 0) {
+    const void* ptrs[] = {q, sink, ring, idx, cbp, rope, workspace, out, lse};
+    for (const void* p : ptrs)
+      if (!p || !aligned16(p)) return LVQ_EINVAL;
+    if (!ctx_len || !coded_len || (split_lse && ((uintptr_t)split_lse & 3u))) return LVQ_EINVAL;
+  }
+  if ((s = check_device()) != LVQ_OK) return s;
+  return cuda_status(launch_decode(g, layer, step, batch, static_cast<const __nv_bfloat16*>(q), ctx_len,
+                                   coded_len, static_cast<const __nv_bfloat16*>(sink),
+                                   static_cast<const __nv_bfloat16*>(ring), idx,
+                                   static_cast<const __nv_bfloat16*>(cbp), rope, num_splits, workspace, out,
+                                   lse, split_lse, dev_status, static_cast<cudaStream_t>(stream)));
+}
+
+lvq_status lvq_dequantize(const lvq_config* cfg, const lvq_layout* lay, int32_t layer, int32_t step,
+                          int32_t req, int32_t kv, const uint8_t* idx, const void* cbp, int32_t tok_begin,
+                          int32_t n_tok, void* out, void* stream) {
+  Geo g;
+  lvq_status s = check_all(cfg, lay, &g);
+  if (s != LVQ_OK) return s;
+  if (layer < 0 || layer >= g.L || step < 0 || step >= g.T || req < 0 || req >= g.B || (kv != 0 && kv != 1) ||
+      tok_begin < 0 || n_tok < 0 || (int64_t)tok_begin + n_tok > (int64_t)g.P * kPage)
+    return LVQ_EINVAL;
+  if (n_tok > 0 && (!idx || !cbp || !out || !aligned16(idx) || !aligned16(cbp) || !aligned16(out)))
+    return LVQ_EINVAL;
+  if ((s = check_device()) != LVQ_OK) return s;
+  return cuda_status(launch_dequantize(g, layer, step, req, kv, idx, static_cast<const __nv_bfloat16*>(cbp),
+                                       tok_begin, n_tok, static_cast<__nv_bfloat16*>(out),
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,226 @@
+"""ctypes binding of liblvq (include/lvq.h), same names as the C ABI.
+
+Argument marshalling only: every step of the codec and the attention runs in
+the library's CUDA kernels.  torch supplies device memory and streams.  If the
+library is missing, or the device is not sm_100, calls raise: there is no
+fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblvq.so")
+
+LVQ_OK, LVQ_EINVAL, LVQ_EUNSUPPORTED, LVQ_ECAPACITY, LVQ_ECUDA, LVQ_ETIMEOUT, LVQ_EDEVICE = range(7)
+
+
+class LvqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class lvq_config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "n_layers", "n_kv_heads", "n_q_heads", "head_dim", "T", "Tc", "G", "K", "n_sink", "n_recent",
+        "page_tokens", "max_batch", "max_ctx", "max_splits")] + [("rope_base", ctypes.c_float)]
+
+
+class lvq_layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "c", "n_groups", "n_blocks", "ring_tokens", "max_pages", "page_bytes", "rope_coarse", "reserved")] + [
+        ("idx_bytes", ctypes.c_size_t), ("idx_strides", ctypes.c_int64 * 8),
+        ("cb_bytes", ctypes.c_size_t), ("cb_strides", ctypes.c_int64 * 7),
+        ("cbp_bytes", ctypes.c_size_t), ("cbp_strides", ctypes.c_int64 * 8),
+        ("cb_norm_bytes", ctypes.c_size_t),
+        ("sink_bytes", ctypes.c_size_t), ("sink_strides", ctypes.c_int64 * 7),
+        ("ring_bytes", ctypes.c_size_t), ("ring_strides", ctypes.c_int64 * 7),
+        ("rope_bytes", ctypes.c_size_t), ("workspace_bytes", ctypes.c_size_t)]
+
+
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_SIGS = {
+    "lvq_cache_layout": [ctypes.POINTER(lvq_config), ctypes.POINTER(lvq_layout)],
+    "lvq_pack_codebooks": [ctypes.POINTER(lvq_config), ctypes.POINTER(lvq_layout), _P, _P, _P, _P],
+    "lvq_rope_table": [ctypes.POINTER(lvq_config), ctypes.POINTER(lvq_layout), _P, _P],
+    "lvq_encode_prefill": [ctypes.POINTER(lvq_config), ctypes.POINTER(lvq_layout), _I32, _I32, _P,
+                           ctypes.c_int64, _I32, _I32, _I32, _I32, _P, _P, _P, _P],
+    "lvq_encode_page": [ctypes.POINTER(lvq_config), ctypes.POINTER(lvq_layout), _I32, _P, _P, _P, _P, _P,
+                        _P, _P],
+    "lvq_decode_attention": [ctypes.POINTER(lvq_config), ctypes.POINTER(lvq_layout), _I32, _I32, _I32, _P,
+                             _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P, _P, _P],
+    "lvq_dequantize": [ctypes.POINTER(lvq_config), ctypes.POINTER(lvq_layout), _I32, _I32, _I32, _I32, _P,
+                       _P, _I32, _I32, _P, _P],
+    "lvq_status_string": [_I32],
+}
+EXPORTED = tuple(_SIGS)
+
+_lib = None
+
+
+def lib():
+    """Loads liblvq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m sub_bit_kv_b200._build`")
+        h = ctypes.CDLL(LIB_PATH)
+        for name, args in _SIGS.items():
+            fn = getattr(h, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_char_p if name == "lvq_status_string" else ctypes.c_int
+        _lib = h
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return lib().lvq_status_string(int(s)).decode()
+
+
+def _check(s: int, where: str):
+    if s != LVQ_OK:
+        raise LvqError(s, where)
+
+
+def make_config(n_layers, n_kv_heads, n_q_heads, head_dim, T, Tc, G, n_sink, n_recent, max_batch, max_ctx,
+                max_splits=64, rope_base=10000.0, K=256, page_tokens=8) -> lvq_config:
+    return lvq_config(n_layers, n_kv_heads, n_q_heads, head_dim, T, Tc, G, K, n_sink, n_recent, page_tokens,
+                      max_batch, max_ctx, max_splits, rope_base)
+
+
+def lvq_cache_layout(cfg: lvq_config) -> lvq_layout:
+    lay = lvq_layout()
+    _check(lib().lvq_cache_layout(ctypes.byref(cfg), ctypes.byref(lay)), "lvq_cache_layout")
+    return lay
+
+
+def _ptr(t: Optional[torch.Tensor], name: str, dtype=None, min_bytes: int = 0, optional=False):
+    if t is None:
+        if optional:
+            return None
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.numel() * t.element_size() < min_bytes:
+        raise ValueError(f"{name} holds {t.numel() * t.element_size()} bytes, needs {min_bytes}")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def lvq_pack_codebooks(cfg, lay, cb, cbp, cb_norm=None, stream=None):
+    _check(lib().lvq_pack_codebooks(
+        ctypes.byref(cfg), ctypes.byref(lay), _ptr(cb, "cb", torch.bfloat16, lay.cb_bytes),
+        _ptr(cbp, "cbp", torch.bfloat16, lay.cbp_bytes),
+        _ptr(cb_norm, "cb_norm", torch.float32, lay.cb_norm_bytes, optional=True), _stream(stream)),
+        "lvq_pack_codebooks")
+
+
+def lvq_rope_table(cfg, lay, rope, stream=None):
+    _check(lib().lvq_rope_table(ctypes.byref(cfg), ctypes.byref(lay), _ptr(rope, "rope", torch.float32,
+                                                                           lay.rope_bytes), _stream(stream)),
+           "lvq_rope_table")
+
+
+def lvq_encode_prefill(cfg, lay, layer, req, kv, tok_begin, n_tok, coded_offset, cb, idx, dev_status,
+                       kv_tok_stride=None, stream=None):
+    """kv: bf16 [2][T][N][Hkv][d] of one layer and request (contiguous)."""
+    if kv.dim() != 5 or kv.shape[0] != 2 or kv.shape[1] != cfg.T:
+        raise ValueError("kv must be [2][T][N][Hkv][d]")
+    n_total = kv.shape[2]
+    stride = kv_tok_stride if kv_tok_stride is not None else kv.shape[3] * kv.shape[4]
+    _check(lib().lvq_encode_prefill(
+        ctypes.byref(cfg), ctypes.byref(lay), layer, req, _ptr(kv, "kv", torch.bfloat16), stride, n_total,
+        tok_begin, n_tok, coded_offset, _ptr(cb, "cb", torch.bfloat16, lay.cb_bytes),
+        _ptr(idx, "idx", torch.uint8, lay.idx_bytes), _ptr(dev_status, "dev_status", torch.int32, 4),
+        _stream(stream)), "lvq_encode_prefill")
+
+
+def lvq_encode_page(cfg, lay, batch, ctx_len, coded_len, ring, cb, idx, dev_status, stream=None):
+    _check(lib().lvq_encode_page(
+        ctypes.byref(cfg), ctypes.byref(lay), batch, _ptr(ctx_len, "ctx_len", torch.int32, 4 * batch),
+        _ptr(coded_len, "coded_len", torch.int32, 4 * batch), _ptr(ring, "ring", torch.bfloat16, lay.ring_bytes),
+        _ptr(cb, "cb", torch.bfloat16, lay.cb_bytes), _ptr(idx, "idx", torch.uint8, lay.idx_bytes),
+        _ptr(dev_status, "dev_status", torch.int32, 4), _stream(stream)), "lvq_encode_page")
+
+
+def lvq_decode_attention(cfg, lay, layer, step, batch, q, ctx_len, coded_len, sink, ring, idx, cbp, rope,
+                         num_splits, workspace, out, lse, dev_status, split_lse=None, stream=None):
+    d = cfg.head_dim
+    _check(lib().lvq_decode_attention(
+        ctypes.byref(cfg), ctypes.byref(lay), layer, step, batch,
+        _ptr(q, "q", torch.bfloat16, 2 * batch * cfg.n_q_heads * d),
+        _ptr(ctx_len, "ctx_len", torch.int32, 4 * batch), _ptr(coded_len, "coded_len", torch.int32, 4 * batch),
+        _ptr(sink, "sink", torch.bfloat16, lay.sink_bytes), _ptr(ring, "ring", torch.bfloat16, lay.ring_bytes),
+        _ptr(idx, "idx", torch.uint8, lay.idx_bytes), _ptr(cbp, "cbp", torch.bfloat16, lay.cbp_bytes),
+        _ptr(rope, "rope", torch.float32, lay.rope_bytes), num_splits,
+        _ptr(workspace, "workspace", torch.float32, lay.workspace_bytes),
+        _ptr(out, "out", torch.float32, 4 * batch * cfg.n_q_heads * d),
+        _ptr(lse, "lse", torch.float32, 4 * batch * cfg.n_q_heads),
+        _ptr(split_lse, "split_lse", torch.float32, 4 * batch * cfg.n_q_heads * (num_splits + 1), optional=True),
+        _ptr(dev_status, "dev_status", torch.int32, 4), _stream(stream)), "lvq_decode_attention")
+
+
+def lvq_dequantize(cfg, lay, layer, step, req, kv, idx, cbp, tok_begin, n_tok, out, stream=None):
+    _check(lib().lvq_dequantize(
+        ctypes.byref(cfg), ctypes.byref(lay), layer, step, req, kv, _ptr(idx, "idx", torch.uint8, lay.idx_bytes),
+        _ptr(cbp, "cbp", torch.bfloat16, lay.cbp_bytes), tok_begin, n_tok,
+        _ptr(out, "out", torch.bfloat16, 2 * n_tok * cfg.n_kv_heads * cfg.head_dim), _stream(stream)),
+        "lvq_dequantize")
+
+
+class CodedCache:
+    """Device buffers of one configuration, allocated with torch to the sizes
+    lvq_cache_layout gives (plumbing: the library itself allocates nothing)."""
+
+    def __init__(self, cfg: lvq_config, device="cuda"):
+        self.cfg = cfg
+        self.lay = lay = lvq_cache_layout(cfg)
+        dev = torch.device(device)
+        self.idx = torch.zeros(lay.idx_bytes, dtype=torch.uint8, device=dev)
+        self.cb = torch.zeros(lay.cb_bytes // 2, dtype=torch.bfloat16, device=dev)
+        self.cbp = torch.zeros(lay.cbp_bytes // 2, dtype=torch.bfloat16, device=dev)
+        self.sink = torch.zeros(lay.sink_bytes // 2, dtype=torch.bfloat16, device=dev)
+        self.ring = torch.zeros(lay.ring_bytes // 2, dtype=torch.bfloat16, device=dev)
+        self.rope = torch.zeros(lay.rope_bytes // 4, dtype=torch.float32, device=dev)
+        self.workspace = torch.zeros(lay.workspace_bytes // 4, dtype=torch.float32, device=dev)
+        self.ctx_len = torch.zeros(cfg.max_batch, dtype=torch.int32, device=dev)
+        self.coded_len = torch.zeros(cfg.max_batch, dtype=torch.int32, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    # shaped views of the caller-owned buffers (layouts from lvq_cache_layout)
+    def cb_view(self):
+        c = self.cfg
+        return self.cb.view(c.n_layers, 2, self.lay.n_blocks, c.n_kv_heads, self.lay.n_groups, 256, c.G)
+
+    def sink_view(self):
+        c = self.cfg
+        return self.sink.view(c.n_layers, 2, c.T, c.max_batch, c.n_kv_heads, c.n_sink, c.head_dim)
+
+    def ring_view(self):
+        c = self.cfg
+        return self.ring.view(c.n_layers, 2, c.T, c.max_batch, c.n_kv_heads, self.lay.ring_tokens, c.head_dim)
+
+    def idx_view(self):
+        c, l = self.cfg, self.lay
+        return self.idx.view(c.n_layers, l.n_blocks, c.max_batch, c.n_kv_heads, l.max_pages, 2, l.n_groups, 8)
+
+    def check_status(self, where="device"):
+        s = int(self.status.item())
+        if s != LVQ_OK:
+            self.status.zero_()
+            raise LvqError(s, where)

@@ -1,0 +1,105 @@
+"""The C-ABI library loads, exports every declared symbol, and its host-side
+layout arithmetic matches the closed forms (CPU only; no compute calls)."""
+import os
+import re
+
+import pytest
+
+from oracle import lvq_oracle as O
+from sub_bit_kv_b200 import lvq, synth
+from tests._helpers import make_cfg
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "lvq.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from sub_bit_kv_b200 import _build
+    _build.build()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:LVQ_API\s+)?(?:lvq_status|const char\*)\s+(lvq_\w+)\s*\(", text, re.M)))
+
+
+def test_exports_every_declared_symbol():
+    names = declared_functions()
+    assert "lvq_decode_attention" in names and "lvq_cache_layout" in names
+    lib = lvq.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(lvq.EXPORTED)
+
+
+def test_status_strings():
+    for s in range(7):
+        assert lvq.status_string(s)
+    assert lvq.status_string(0) == "ok"
+
+
+@pytest.mark.parametrize("name", list(synth.WORKLOADS))
+def test_layout_closed_forms(name):
+    w = synth.WORKLOADS[name]
+    cfg = make_cfg(w)
+    lay = lvq.lvq_cache_layout(cfg)
+    c, ng, nblk = O.geometry(w.head_dim, w.T, w.Tc, w.G)
+    assert (lay.c, lay.n_groups, lay.n_blocks) == (c, ng, nblk)
+    assert lay.page_bytes == 2 * ng * 8
+    assert lay.ring_tokens == w.n_recent + 8
+    # code bytes per token, head and K/V: one row of n_g bytes per block ("one index row per Tc block")
+    per_token = lay.idx_bytes / (cfg.n_layers * cfg.max_batch * cfg.n_kv_heads * lay.max_pages * 8 * 2)
+    assert per_token == nblk * ng
+    # bits per cached element = 8/G
+    assert per_token * 8 / (w.T * w.head_dim) == 8 / w.G
+    assert lay.cb_bytes == cfg.n_layers * 2 * nblk * cfg.n_kv_heads * ng * 256 * w.G * 2
+    assert lay.cbp_bytes == lay.cb_bytes
+    assert list(lay.idx_strides)[-3:] == [ng * 8, 8, 1]
+    assert list(lay.ring_strides)[-2:] == [w.head_dim, 1]
+
+
+def test_ouro_row_bytes():
+    rows = {}
+    for name, want in (("ouro14_g16_32k", (1, 32)), ("ouro14_g32_b32", (1, 16)), ("ouro14_tc2_64k", (2, 16))):
+        lay = lvq.lvq_cache_layout(make_cfg(synth.WORKLOADS[name]))
+        rows[name] = (lay.n_blocks, lay.n_groups)
+        assert rows[name] == want
+    # index storage for 24 layers x 16 heads at 32K context, B = 1: 24.6 KB per token
+    w = synth.WORKLOADS["ouro14_g16_32k"]
+    per_tok = w.n_layers * w.n_kv_heads * 2 * 32
+    assert per_tok == 24576
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("Tc", 3, lvq.LVQ_EINVAL),           # Tc does not divide T = 4
+    ("G", 18, lvq.LVQ_EINVAL),           # Tc = 4 does not divide G
+    ("K", 128, lvq.LVQ_EUNSUPPORTED),
+    ("page_tokens", 16, lvq.LVQ_EUNSUPPORTED),
+    ("head_dim", 96, lvq.LVQ_EUNSUPPORTED),
+    ("n_q_heads", 24, lvq.LVQ_EINVAL),    # not a multiple of 16 KV heads
+    ("max_splits", 0, lvq.LVQ_EINVAL),
+    ("n_layers", 0, lvq.LVQ_EINVAL),
+])
+def test_invalid_configs_rejected(field, value, status):
+    cfg = make_cfg(synth.WORKLOADS["ouro14_g16_32k"])
+    setattr(cfg, field, value)
+    with pytest.raises(lvq.LvqError) as e:
+        lvq.lvq_cache_layout(cfg)
+    assert e.value.status == status
+
+
+def test_layout_mismatch_is_rejected_before_any_device_work():
+    """A caller's layout that does not match its config fails with EINVAL on the host."""
+    import ctypes
+    w = synth.WORKLOADS["tiny"]
+    cfg = make_cfg(w)
+    lay = lvq.lvq_cache_layout(cfg)
+    lay.idx_bytes += 1
+    st = lvq.lib().lvq_rope_table(ctypes.byref(cfg), ctypes.byref(lay), None, None)
+    assert st == lvq.LVQ_EINVAL
+    lay = lvq.lvq_cache_layout(cfg)
+    st = lvq.lib().lvq_rope_table(ctypes.byref(cfg), ctypes.byref(lay), None, None)
+    assert st == lvq.LVQ_EINVAL          # null table pointer
+    st = lvq.lib().lvq_decode_attention(ctypes.byref(cfg), ctypes.byref(lay), 0, 4, 1, *([None] * 8), 1,
+                                        None, None, None, None, None, None)
+    assert st == lvq.LVQ_EINVAL          # step 4 out of range for T = 4
