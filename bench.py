@@ -202,8 +202,8 @@ def build_cache(w, lvq, synth, torch, extra_tokens: int, device, request_seed: i
 
 
 def choose_splits(w, n_sm: int) -> int:
-    # about two CTAs per SM over the H kv heads: splits * H ~ 2 * SMs
-    return max(1, min(128, round(2 * n_sm / (w.batch * w.n_q_heads))))
+    # one CTA per SM: splits * heads * requests ~ SMs
+    return max(1, min(128, n_sm // (w.batch * w.n_q_heads)))
 
 
 def decode_bytes_per_launch(w, lay, coded: int, recent: int) -> int:
@@ -259,7 +259,7 @@ def gpu_arm(args):
         lvq.lvq_encode_page(cfg, lay, B, cache.ctx_len, cache.coded_len, cache.ring, cache.cb, cache.idx,
                             cache.status, stream=stream)
 
-    launches_per_step = TOKENS_PER_STEP * NL * 2 + 2
+    launches_per_step = TOKENS_PER_STEP * NL + 2
     stream = torch.cuda.Stream(device)
     # one eager step to check everything runs, then capture the step
     with torch.cuda.stream(stream):
@@ -391,7 +391,7 @@ def gpu_arm(args):
                    "num_splits": ns, "tokens_per_step": TOKENS_PER_STEP,
                    "l2": "inputs larger than L2 (3.5 GB of codes per token)", "parallelism": f"replicas{world}"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": None, "kernel": "decode_split_kernel<128,4> + merge",
+                     "frac": achieved / hbm_peak, "traffic": None, "kernel": "decode_kernel<128,4>",
                      "peak_kind": peak_kind, "bytes_per_launch": bpl, "launch_ms": per_call_ms},
         "code_stream_GBps": code_stream,
         "cpu_baseline": cb,

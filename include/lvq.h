@@ -85,7 +85,7 @@ typedef struct {
   int32_t page_tokens;  /* must be 8 */
   int32_t max_batch;    /* requests the cache holds */
   int32_t max_ctx;      /* longest context (tokens, including the query) */
-  int32_t max_splits;   /* largest num_splits lvq_decode_attention accepts */
+  int32_t max_splits;   /* largest num_splits lvq_decode_attention accepts (<= 256) */
   float rope_base;      /* RoPE base (10000 for the Ouro-shaped workloads) */
 } lvq_config;
 
@@ -127,7 +127,9 @@ typedef struct {
   /* fp32 RoPE tables: coarse [rope_coarse][d/2] (cos, sin) of 8k*theta_f,
    * then fine [8][d/2] (cos, sin) of r*theta_f.  Written by lvq_rope_table. */
   size_t rope_bytes;
-  /* fp32 split partials, [B][Hq][max_splits + 1][d + 2] */
+  /* scratch of lvq_decode_attention: fp32 split partials
+   * [B][Hq][max_splits + 1][d + 2], then int32 merge counters [B][Hq].  Zero
+   * it once before first use; every call leaves the counters at zero. */
   size_t workspace_bytes;
 } lvq_layout;
 
@@ -196,7 +198,9 @@ LVQ_API lvq_status lvq_encode_page(const lvq_config* cfg, const lvq_layout* lay,
  *   num_splits: coded tokens are cut into num_splits ranges, split j covering
  *     [j*chunk, min(L, (j+1)*chunk)), chunk = ceil(L/num_splits) rounded up to
  *     a multiple of 32; the bf16 tokens are one more partial.
- *   workspace: fp32 scratch of lay->workspace_bytes.
+ *   workspace: scratch of lay->workspace_bytes, zeroed once before first use
+ *     (its merge counters return to zero at the end of every call).  Calls
+ *     that share a workspace must not overlap on the GPU.
  *   out: device fp32 [batch][Hq][d]; lse: device fp32 [batch][Hq], natural log
  *     of the softmax denominator (scores scaled by 1/sqrt(d)).
  *   split_lse: NULL, or device fp32 [batch][Hq][num_splits + 1] receiving each

@@ -25,7 +25,7 @@ lvq_status check_cfg(const lvq_config* c) {
   if (c->head_dim % cc || (c->head_dim / cc) % 2) return LVQ_EINVAL;
   if (c->K != kEntries || c->page_tokens != kPage) return LVQ_EUNSUPPORTED;
   if (!decode_supported(c->head_dim, cc) || !encode_supported(c->G, cc)) return LVQ_EUNSUPPORTED;
-  if (c->max_splits > 1024 || c->max_ctx > (1 << 28)) return LVQ_EUNSUPPORTED;
+  if (c->max_splits > 256 || c->max_ctx > (1 << 28)) return LVQ_EUNSUPPORTED;
   return LVQ_OK;
 }
 
@@ -37,7 +37,7 @@ Geo make_geo(const lvq_config* c) {
   const int max_coded = c->max_ctx > c->n_sink ? c->max_ctx - c->n_sink : 0;
   g.P = max_coded > 0 ? (max_coded + kPage - 1) / kPage : 1;
   g.B = c->max_batch; g.max_ctx = c->max_ctx; g.max_splits = c->max_splits;
-  g.RC = (c->max_ctx + kPage - 1) / kPage + 16;
+  g.RC = max((c->max_ctx + kPage - 1) / kPage, 64) + 16;   // rows cover offsets up to 512 positions
   g.page_bytes = 2 * g.ng * kPage;
   return g;
 }
@@ -68,7 +68,7 @@ void fill_layout(const Geo& g, lvq_layout* o) {
   for (int i = 6; i >= 0; --i) { o->ring_strides[i] = st; st *= rdims[i]; }
   o->ring_bytes = (size_t)st * 2;
   o->rope_bytes = (size_t)(g.RC + kPage) * (g.d / 2) * 2 * 4;
-  o->workspace_bytes = (size_t)g.B * g.Hq * (g.max_splits + 1) * (g.d + 2) * 4;
+  o->workspace_bytes = (size_t)g.B * g.Hq * (g.max_splits + 1) * (g.d + 2) * 4 + (size_t)g.B * g.Hq * 4;
 }
 
 // Re-derives the layout and checks the caller's copy matches it.
