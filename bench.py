@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--splits", type=int, default=0, help="split count (0: choose)")
     ap.add_argument("--no-encode", action="store_true", help="skip the prefill-encode measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--profile", default="", choices=["", "decode", "encode"],
+                    help="build the workload, run 3 launches of one kernel and exit (for ncu captures)")
     return ap.parse_args()
 
 
@@ -202,8 +204,8 @@ def build_cache(w, lvq, synth, torch, extra_tokens: int, device, request_seed: i
 
 
 def choose_splits(w, n_sm: int) -> int:
-    # one CTA per SM: splits * heads * requests ~ SMs
-    return max(1, min(128, n_sm // (w.batch * w.n_q_heads)))
+    # one CTA per SM: (splits + 1 bf16 CTA) * heads * requests <= SMs
+    return max(1, min(128, n_sm // (w.batch * w.n_q_heads) - 1))
 
 
 def decode_bytes_per_launch(w, lay, coded: int, recent: int) -> int:
@@ -213,6 +215,20 @@ def decode_bytes_per_launch(w, lay, coded: int, recent: int) -> int:
     bf16 = (min(w.n_sink, coded + recent) + recent) * w.n_kv_heads * 2 * w.head_dim * 2
     qo = w.n_q_heads * w.head_dim * (2 + 4) + w.n_q_heads * 4
     return idx + slices + bf16 + qo
+
+
+def profile_encode(lvq, synth, torch, device):
+    """One Ouro-2.6B-shaped layer (32768 tokens), encoded 3 times."""
+    wc = synth.WORKLOADS["ouro26_prefill_32k"]
+    cfg4 = lvq.make_config(1, wc.n_kv_heads, wc.n_q_heads, wc.head_dim, wc.T, wc.Tc, wc.G, 0, 0, 1, wc.ctx,
+                           max_splits=1, rope_base=wc.rope_base)
+    c4 = lvq.CodedCache(cfg4, device)
+    c4.cb_view()[0] = synth.codebooks(wc, 0, device=device)
+    kv4 = synth.loop_kv(wc, 0, wc.ctx, stream="coded", device=device)
+    for _ in range(3):
+        lvq.lvq_encode_prefill(cfg4, c4.lay, 0, 0, kv4, 0, wc.ctx, 0, c4.cb, c4.idx, c4.status)
+    torch.cuda.synchronize()
+    c4.check_status("profile encode")
 
 
 def gpu_arm(args):
@@ -234,6 +250,9 @@ def gpu_arm(args):
         dist.barrier()
     lvq.lib()
 
+    if args.profile == "encode":
+        profile_encode(lvq, synth, torch, device)
+        return
     w = synth.WORKLOADS[WORKLOAD]
     replays = 2 * args.steps + args.warmup + 3          # every graph replay adds 8 tokens
     cfg, cache = build_cache(w, lvq, synth, torch, TOKENS_PER_STEP * (replays + 4), device, rank)
@@ -241,6 +260,17 @@ def gpu_arm(args):
     n_sm = torch.cuda.get_device_properties(device).multi_processor_count
     ns = args.splits or choose_splits(w, n_sm)
     B, Hq, d = w.batch, w.n_q_heads, w.head_dim
+    if args.profile == "decode":
+        q = torch.randn(B, Hq, d, device=device).to(torch.bfloat16)
+        o = torch.empty(B, Hq, d, device=device)
+        l = torch.empty(B, Hq, device=device)
+        for layer in range(3):
+            lvq.lvq_decode_attention(cfg, lay, layer, 0, B, q, cache.ctx_len, cache.coded_len, cache.sink,
+                                     cache.ring, cache.idx, cache.cbp, cache.rope, ns, cache.workspace, o, l,
+                                     cache.status)
+        torch.cuda.synchronize()
+        cache.check_status("profile")
+        return
     NL = w.n_layers * w.T                                            # attentions per token
     q_all = torch.randn(TOKENS_PER_STEP, w.T, w.n_layers, B, Hq, d, device=device,
                         generator=synth.generator(device, w.seed, "bench-q", rank)).to(torch.bfloat16)
@@ -373,7 +403,7 @@ def gpu_arm(args):
         enc_ms = a.elapsed_time(b_) / 3
         vectors = wc.ctx * wc.n_kv_heads * 2 * (wc.head_dim // (wc.G // wc.Tc)) * (wc.T // wc.Tc)
         enc = {"vectors_per_s": vectors / (enc_ms / 1e3), "ms_per_layer": enc_ms,
-               "workload": "ouro26_prefill_32k (one of 48 layers)", "kernel": "encode_prefill (fp64 direct form)"}
+               "workload": "ouro26_prefill_32k (one of 48 layers)", "kernel": "encode_tc (tcgen05 distance GEMM + argmin)"}
         del kv4, c4
 
     if rank != 0:

@@ -26,6 +26,7 @@ lvq_status check_cfg(const lvq_config* c) {
   if (c->K != kEntries || c->page_tokens != kPage) return LVQ_EUNSUPPORTED;
   if (!decode_supported(c->head_dim, cc) || !encode_supported(c->G, cc)) return LVQ_EUNSUPPORTED;
   if (c->max_splits > 256 || c->max_ctx > (1 << 28)) return LVQ_EUNSUPPORTED;
+  if (c->n_sink + c->n_recent + kPage > decode_bf16_capacity(c->head_dim, cc)) return LVQ_EUNSUPPORTED;
   return LVQ_OK;
 }
 
@@ -159,6 +160,13 @@ lvq_status lvq_encode_prefill(const lvq_config* cfg, const lvq_layout* lay, int3
   if (n_tok > 0 && (!kv || !cb || !idx || !aligned16(kv) || !aligned16(cb) || !aligned16(idx)))
     return LVQ_EINVAL;
   if ((s = check_device()) != LVQ_OK) return s;
+  // tensor-core encoder where its tiles fit (c in {4, 8}, 16-byte token rows); the fp64
+  // direct-form encoder otherwise.  Both return the exact nearest entry.
+  if (encode_tc_supported(g.G, g.c) && kv_tok_stride % 8 == 0)
+    return cuda_status(launch_encode_tc(g, layer, req, static_cast<const __nv_bfloat16*>(kv), kv_tok_stride,
+                                        kv_tokens, tok_begin, n_tok, coded_offset,
+                                        static_cast<const __nv_bfloat16*>(cb), idx, dev_status,
+                                        static_cast<cudaStream_t>(stream)));
   return cuda_status(launch_encode_prefill(g, layer, req, static_cast<const __nv_bfloat16*>(kv), kv_tok_stride,
                                            kv_tokens, tok_begin, n_tok, coded_offset,
                                            static_cast<const __nv_bfloat16*>(cb), idx, dev_status,

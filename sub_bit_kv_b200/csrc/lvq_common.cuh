@@ -112,5 +112,10 @@ cudaError_t launch_decode(const Geo& g, int layer, int step, int batch, const __
                           const __nv_bfloat16* cbp, const float* rope, int num_splits, float* ws,
                           float* out, float* lse, float* split_lse, int32_t* st, cudaStream_t s);
 bool decode_supported(int d, int c);
+int decode_bf16_capacity(int d, int c);
+bool encode_tc_supported(int G, int c);
+cudaError_t launch_encode_tc(const Geo& g, int layer, int req, const __nv_bfloat16* kv, int64_t tok_stride,
+                             int kv_tokens, int tok_begin, int n_tok, int coded_offset,
+                             const __nv_bfloat16* cb, uint8_t* idx, int32_t* st, cudaStream_t s);
 bool encode_supported(int G, int c);
 }  // namespace lvq

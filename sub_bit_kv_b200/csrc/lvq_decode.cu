@@ -27,8 +27,10 @@
 //    sum_k H[k][g] * V_slice[k][g][e].  Weights use a reference maximum fixed
 //    per split, raised (and H rescaled) only if a chunk's maximum exceeds it
 //    by 2^16;
-//  * the last split's CTA also computes the bf16 tokens' partial (sink and
-//    recent window) with an online softmax;
+//  * CTA ns (one more per request and head) computes the bf16 tokens'
+//    partial: sink and recent window staged in shared memory by bulk copies,
+//    scores with 4 threads per token, one softmax, P.V with a thread per
+//    channel;
 //  * the last CTA of a (request, head) to finish merges all partials by LSE
 //    (a counter in the workspace, reset by that CTA).
 #include "lvq_common.cuh"
@@ -170,7 +172,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(
   chunk = (chunk + 31) & ~31;
   const int n0 = bad ? 0 : min(Lc, j * chunk), n1 = bad ? 0 : min(Lc, n0 + chunk);
   const bool do_coded = n0 < n1;
-  const bool do_bf16 = !bad && j == ns - 1;
 
   // ---- start the bulk copies: key slice, then the first two chunks of pages
   const uint32_t bar0 = smem_addr(&bars[0]);
@@ -356,18 +357,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(
   }
 
   // ---- coded partial: o[e] = sum_k H[k][g] V[k][g][e mod c]
-  {
+  if (j < ns) {
     const float l_tot = block_reduce<false>(l_acc, red);
     constexpr int NKQ = kDecThreads / D;
     const int e = tid % D, kq = tid / D, grp = e / C, ee = e % C;
     float o = 0.f;
     if (do_coded) {
-      const __nv_bfloat16* Vs = cbp + cbp_slice_off(g, layer, 1, blk, h, s);
+      const __nv_bfloat16* Vs = cbp + cbp_slice_off(g, layer, 1, blk, h, s) + (size_t)grp * C + ee;
+#pragma unroll 8
       for (int k = kq; k < kEntries; k += NKQ) {
         float hsum = 0.f;
 #pragma unroll
         for (int t2 = 0; t2 < TPV; ++t2) hsum += Hs[(k * TPV + t2) * NG + grp];
-        if (hsum != 0.f) o = fmaf(hsum, __bfloat162float(Vs[((size_t)k * NG + grp) * C + ee]), o);
+        o = fmaf(hsum, __bfloat162float(Vs[(size_t)k * D]), o);
       }
     }
     sc[tid] = o;
@@ -380,84 +382,92 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(
     store_partial(part, D, oe, tid < D ? tid : -1, do_coded ? m_ref : -INFINITY, do_coded ? l_tot : 0.f);
   }
 
-  // ---- bf16 partial (sink and recent window), in the last split's CTA
-  if (do_bf16) {
-    constexpr int RF = F / 32;
-    float2 z[RF];
-#pragma unroll
-    for (int r = 0; r < RF; ++r) z[r] = zq[lane + 32 * r];
-    float m = -INFINITY, l = 0.f, olo[RF], ohi[RF];
-#pragma unroll
-    for (int r = 0; r < RF; ++r) { olo[r] = 0.f; ohi[r] = 0.f; }
-    const int nb = S_eff + recent;
-    for (int i = warp; i < nb; i += kDecWarps) {
-      int pos;
-      const __nv_bfloat16 *kp, *vp;
-      if (i < S_eff) {
-        pos = i;
-        kp = sink + sink_off(g, layer, 0, step, b, h, i);
-        vp = sink + sink_off(g, layer, 1, step, b, h, i);
-      } else {
-        pos = g.S + Lc + (i - S_eff);
-        const int slot = (pos - g.S) % g.R;
-        kp = ring + ring_off(g, layer, 0, step, b, h, slot);
-        vp = ring + ring_off(g, layer, 1, step, b, h, slot);
+  // ---- CTA ns: the bf16 partial (sink tokens and recent window)
+  if (j == ns) {
+    float* pb = ws + (slot_base + ns) * (D + 2);
+    const int nb = bad ? 0 : S_eff + recent;
+    // stage sink K/V and the whole recent-window ring K/V for (layer, step, b, h)
+    __nv_bfloat16* Kb = reinterpret_cast<__nv_bfloat16*>(smem);                 // [S + R][D]
+    __nv_bfloat16* Vb = Kb + (size_t)(g.S + g.R) * D;                            // [S + R][D]
+    bool ok = true;
+    if (nb > 0) {
+      const uint32_t barb = smem_addr(&bars[0]);
+      if (tid == 0) {
+        mbar_init(barb, 1);
+        fence_mbar_init();
+        const uint32_t sb = (uint32_t)S_eff * D * 2, rb = (uint32_t)g.R * D * 2;
+        mbar_expect_tx(barb, 2 * (sb + rb));
+        if (sb) {
+          bulk_g2s(smem_addr(Kb), sink + sink_off(g, layer, 0, step, b, h, 0), sb, barb);
+          bulk_g2s(smem_addr(Vb), sink + sink_off(g, layer, 1, step, b, h, 0), sb, barb);
+        }
+        bulk_g2s(smem_addr(Kb + (size_t)g.S * D), ring + ring_off(g, layer, 0, step, b, h, 0), rb, barb);
+        bulk_g2s(smem_addr(Vb + (size_t)g.S * D), ring + ring_off(g, layer, 1, step, b, h, 0), rb, barb);
       }
-      float ps = 0.f;
-#pragma unroll
-      for (int r = 0; r < RF; ++r) {
-        const int f = lane + 32 * r;
-        const float2 w = cmul(z[r], cconj(rope_at(rope, g.RC, F, pos, f)));
-        ps += w.x * __bfloat162float(kp[f]) + w.y * __bfloat162float(kp[f + F]);
-      }
-      const float s2 = warp_sum(ps);
-      const float mn = fmaxf(m, s2);
-      const float alpha = exp2f(m - mn), pp = exp2f(s2 - mn);
-      l = l * alpha + pp;
-#pragma unroll
-      for (int r = 0; r < RF; ++r) {
-        const int f = lane + 32 * r;
-        olo[r] = olo[r] * alpha + pp * __bfloat162float(vp[f]);
-        ohi[r] = ohi[r] * alpha + pp * __bfloat162float(vp[f + F]);
-      }
-      m = mn;
+      __syncthreads();
+      ok = !__syncthreads_or(!mbar_wait(barb, 0, kWaitIters));
+      if (!ok && tid == 0) set_status(st, LVQ_ETIMEOUT);
     }
-    __syncthreads();   // Hs and sc are free: reuse for the warps' partials
-    if (lane == 0) { sc[warp] = m; sc[kDecWarps + warp] = l; }
-#pragma unroll
-    for (int r = 0; r < RF; ++r) {
-      Hs[warp * D + lane + 32 * r] = olo[r];
-      Hs[warp * D + F + lane + 32 * r] = ohi[r];
+    // scores: 4 threads per token, each a quarter of the frequencies
+    constexpr int FQ = F / 4;
+    for (int i0 = 0; i0 < nb && ok; i0 += kDecThreads / 4) {
+      const int i = i0 + tid / 4, qf = tid % 4;
+      float part_s = 0.f;
+      if (i < nb) {
+        int pos, row;
+        if (i < S_eff) { pos = i; row = i; }
+        else { pos = g.S + Lc + (i - S_eff); row = g.S + (pos - g.S) % g.R; }
+        const __nv_bfloat16* kr = Kb + (size_t)row * D;
+#pragma unroll 4
+        for (int f = qf * FQ; f < (qf + 1) * FQ; ++f) {
+          const float2 w = cmul(zq[f], cconj(rope_at(rope, g.RC, F, pos, f)));
+          part_s = fmaf(w.x, __bfloat162float(kr[f]), part_s);
+          part_s = fmaf(w.y, __bfloat162float(kr[f + F]), part_s);
+        }
+      }
+      part_s += __shfl_xor_sync(0xffffffffu, part_s, 1);
+      part_s += __shfl_xor_sync(0xffffffffu, part_s, 2);
+      if (i < nb && qf == 0) sc[i] = part_s;
     }
     __syncthreads();
-    float M = -INFINITY;
-    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, sc[w]);
-    float* pb = ws + (slot_base + ns) * (D + 2);
+    float mloc = -INFINITY;
+    for (int i = tid; i < nb && ok; i += kDecThreads) mloc = fmaxf(mloc, sc[i]);
+    const float M = block_reduce<true>(mloc, red);
+    float lloc = 0.f;
+    for (int i = tid; i < nb && ok; i += kDecThreads) {
+      const float p = exp2f(sc[i] - M);
+      sc[i] = p;
+      lloc += p;
+    }
+    const float Lb = block_reduce<false>(lloc, red);     // block_reduce syncs: sc holds the weights
+    constexpr int NTS = kDecThreads / D;
+    const int e = tid % D, ts = tid / D;
+    float o = 0.f;
+    for (int i = ts; i < nb && ok; i += NTS) {
+      const int row = i < S_eff ? i : g.S + (Lc + (i - S_eff)) % g.R;
+      o = fmaf(sc[i], __bfloat162float(Vb[(size_t)row * D + e]), o);
+    }
+    __syncthreads();
+    Hs[ts * D + e] = o;    // after the barrier nothing reads the staged tokens any more
+    __syncthreads();
     if (tid < D) {
-      float o = 0.f;
-      if (M != -INFINITY)
-        for (int w = 0; w < kDecWarps; ++w)
-          if (sc[w] != -INFINITY) o += exp2f(sc[w] - M) * Hs[w * D + tid];
-      pb[tid] = o;
+      float oe = 0.f;
+#pragma unroll
+      for (int k2 = 0; k2 < NTS; ++k2) oe += Hs[k2 * D + tid];
+      pb[tid] = oe;
     }
     if (tid == 0) {
-      float L = 0.f;
-      if (M != -INFINITY)
-        for (int w = 0; w < kDecWarps; ++w)
-          if (sc[w] != -INFINITY) L += exp2f(sc[w] - M) * sc[kDecWarps + w];
-      pb[D] = M;
-      pb[D + 1] = L;
+      const bool any = ok && nb > 0;
+      pb[D] = any ? M : -INFINITY;
+      pb[D + 1] = any ? Lb : 0.f;
     }
-  } else if (j == ns - 1 && tid < D + 2) {
-    float* pb = ws + (slot_base + ns) * (D + 2);
-    pb[tid] = tid == D ? -INFINITY : 0.f;
   }
 
   // ---- the last CTA of this (request, head) merges the ns + 1 partials
   __threadfence();
   __syncthreads();
   __shared__ int last;
-  if (tid == 0) last = atomicAdd(&counters[(size_t)b * g.Hq + hq], 1) == ns - 1;
+  if (tid == 0) last = atomicAdd(&counters[(size_t)b * g.Hq + hq], 1) == ns;
   __syncthreads();
   if (!last) return;
   __threadfence();
@@ -507,10 +517,24 @@ static cudaError_t decode_as(const Geo& g, int layer, int step, int batch, const
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < kMaxDevices) attr_set[dev] = true;
   }
-  dim3 grid(ns, g.Hq, batch);
+  dim3 grid(ns + 1, g.Hq, batch);
   decode_kernel<D, C><<<grid, kDecThreads, Dec<D, C>::SMEM, s>>>(
       g, layer, step, q, ctx_len, coded_len, sink, ring, idx, cbp, rope, ns, ws, out, lse, split_lse, st);
   return cudaGetLastError();
+}
+
+// bf16 tokens (sink + ring slots) the bf16-partial CTA can stage: K and V must
+// fit below the score buffer.
+template <int D, int C>
+static int bf16_capacity_as() { return Dec<D, C>::OFF_SC / (4 * D); }
+
+int decode_bf16_capacity(int d, int c) {
+  if (d == 128 && c == 4) return bf16_capacity_as<128, 4>();
+  if (d == 128 && c == 8) return bf16_capacity_as<128, 8>();
+  if (d == 128 && c == 16) return bf16_capacity_as<128, 16>();
+  if (d == 64 && c == 4) return bf16_capacity_as<64, 4>();
+  if (d == 64 && c == 8) return bf16_capacity_as<64, 8>();
+  return 0;
 }
 
 bool decode_supported(int d, int c) {

@@ -1,0 +1,448 @@
+// Prefill encoder on the 5th-generation tensor cores (tcgen05, TMEM).
+//
+// "LoopVQ summary", section "premises and limits": prefill keeps each step's
+// keys and values until the last step, then computes the codebook distances
+// with a matrix multiply and encodes.  Section "how it differs": the code is
+// the single nearest entry of the joint vector.
+//
+// For a tile of 128 joint vectors X (one codebook) the tensor core computes
+//   D[m][k] = ||C_k||^2 - 2 X_m . C_k          (k = 0..255)
+// as one UMMA (M = 128, N = 256) whose K dimension holds the G vector
+// elements and three extra columns: A = [X | 1 1 1 | 0...],
+// B_k = [-2 C_k | n1 n2 n3 | 0...] with n1 + n2 + n3 = ||C_k||^2 split into
+// bf16 parts.  bf16 products are exact and the tensor core accumulates in
+// fp32 in TMEM.  ||X||^2 is left out: it does not change the argmin.
+//
+// Exactness: with eps = 2^-14 (||X||^2 + max_k ||C_k||^2), every entry whose
+// exact distance is the minimum has D <= min(D) + eps.  The epilogue finds
+// min(D), then the set of entries with D <= min(D) + eps.  A single candidate
+// is the exact nearest entry; several (a near-tie) are rescored in fp64 in the
+// direct form sum_j (X_j - C_kj)^2 -- exact for bf16 inputs -- lowest index on
+// ties.  So every code equals the fp64 brute-force answer.
+//
+// CTA: 256 threads, one per SM (it allocates all 512 TMEM columns).  Work items
+// are (K/V, block, head, 16-channel span) x 1024-token ranges.  The raw input
+// tile [Tc][128 tokens][16 channels] arrives by TMA (no multicast) into a
+// 2-stage ring; the 16 channels hold 16/c groups.  Two sets of 4 warps (one
+// per TMEM lane quadrant) each own 256 TMEM columns and alternate over the
+// groups: build the group's A tile, issue its UMMA, and run the argmin
+// epilogue, so one set's epilogue overlaps the other set's MMA.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "lvq_common.cuh"
+
+namespace lvq {
+
+namespace tc {
+
+constexpr int kThreads = 256;
+constexpr int kRows = 128;          // UMMA M
+constexpr int kTileTokens = 128;
+constexpr int kItemTokens = 1024;   // tokens per work item (8 tiles)
+constexpr int kSpan = 16;           // channels per item (TMA box x: 32 bytes)
+constexpr int kRawStages = 2;
+
+template <int G, int C>
+struct Enc {
+  static constexpr int TC = G / C;            // steps per block
+  static constexpr int NGC = kSpan / C;       // groups per item
+  static constexpr int KP = G + 16;           // padded K: G elements, 3 bias columns, zeros
+  static constexpr int KSTEPS = KP / 16;
+  static constexpr int SBO = KP * 16;         // bytes between 8-row core-matrix groups
+  static constexpr int A_TILE = kRows * KP * 2;
+  static constexpr int B_TILE = kEntries * KP * 2;
+  static constexpr int RAW = TC * kTileTokens * kSpan * 2;
+  static constexpr int OFF_B = 0;
+  static constexpr int OFF_A = OFF_B + NGC * B_TILE;
+  static constexpr int OFF_RAW = OFF_A + NGC * A_TILE;
+  static constexpr int OFF_NMAX = OFF_RAW + kRawStages * RAW;
+  static constexpr int OFF_BAR = OFF_NMAX + 16 * 4;
+  static constexpr int OFF_TMEM = OFF_BAR + 8 * (kRawStages + 2);
+  // + alignment slack; at least 120 KB so that one CTA (holding all of TMEM) fits per SM
+  static constexpr int SMEM = (OFF_TMEM + 16 + 1024) > 120 * 1024 ? (OFF_TMEM + 16 + 1024) : 120 * 1024;
+  static_assert(NGC == 2 || NGC == 4, "two MMA sets alternate over the item's groups");
+  static_assert(KP % 16 == 0, "K steps");
+};
+
+// K-major, no-swizzle UMMA shared-memory descriptor: core matrices of 8 rows x
+// 16 bytes, the two K-adjacent core matrices LBO = 128 bytes apart, 8-row
+// groups SBO bytes apart; version 1 (sm_100).
+__device__ inline uint64_t smem_desc(uint32_t addr, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3fff) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)(sbo >> 4) << 32) |
+         (1ull << 46);
+}
+
+// kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, both
+// K-major, N = 256, M = 128.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((256u >> 3) << 17) | ((128u >> 4) << 24);
+
+// byte offset of element (row, k) of a K-major no-swizzle tile
+__device__ inline uint32_t kmaj_off(int row, int k, int sbo) {
+  return (row & 7) * 16 + (row >> 3) * sbo + (k >> 3) * 128 + (k & 7) * 2;
+}
+
+__device__ inline void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+      :: "r"(dst), "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar) : "memory");
+}
+
+__device__ inline void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ inline void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ inline void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ inline void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(n) : "memory"); }
+
+__device__ inline void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
+      :: "r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
+}
+
+__device__ inline void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" :: "r"(bar)
+               : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane
+__device__ inline void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ inline float fmin3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+template <int G, int C>
+__global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
+    const __grid_constant__ CUtensorMap tmap, Geo g, int layer, int req, int tok_begin, int n_tok,
+    int coded_offset, const __nv_bfloat16* __restrict__ cb, uint8_t* __restrict__ idx, int32_t* st) {
+  using X = Enc<G, C>;
+  constexpr int TC = X::TC, NGC = X::NGC, KP = X::KP, SBO = X::SBO;
+  extern __shared__ unsigned char smem_raw[];
+  // 1024-byte alignment of the dynamic shared memory base
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* Bt = smem + X::OFF_B;
+  unsigned char* At = smem + X::OFF_A;
+  unsigned char* raw = smem + X::OFF_RAW;
+  float* nmax_s = reinterpret_cast<float*>(smem + X::OFF_NMAX);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + X::OFF_BAR);  // [0..1] raw stages, [2..3] MMA sets
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + X::OFF_TMEM);
+  volatile int* fail_s = reinterpret_cast<volatile int*>(smem + X::OFF_TMEM + 4);   // per MMA set
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int set = tid / kRows;            // MMA set: warps 0-3 or 4-7
+  const int row = tid % kRows;            // TMEM lane = tile row = token of the tile
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" :: "r"(smem_addr(tmem_slot))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (tid == 0) {
+    for (int i = 0; i < kRawStages + 2; ++i) mbar_init(smem_addr(&bars[i]), 1);
+    fence_mbar_init();
+    fail_s[0] = 0;
+    fail_s[1] = 0;
+  }
+  // zero the A tiles once: the columns past G + 3 stay zero
+  for (int i = tid; i < NGC * X::A_TILE / 16; i += kThreads)
+    reinterpret_cast<uint4*>(At)[i] = make_uint4(0, 0, 0, 0);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t tmem_set = tmem_base + (uint32_t)(set * 256);
+  const uint32_t lane_addr = ((uint32_t)(32 * (warp & 3))) << 16;
+
+  const int n_spans = g.d / kSpan;
+  const int n_sets = 2 * g.nblk * g.H * n_spans;
+  const int n_ranges = (n_tok + kItemTokens - 1) / kItemTokens;
+  const long n_items = (long)n_sets * n_ranges;
+
+  uint32_t raw_phase[kRawStages] = {0, 0};
+  uint32_t mma_phase = 0;
+  int tile_counter = 0;     // tiles processed by this CTA (drives the raw ring)
+  bool failed = false;
+
+  for (long item = blockIdx.x; item < n_items && !failed; item += gridDim.x) {
+    int cs = (int)(item / n_ranges);
+    const int range = (int)(item % n_ranges);
+    const int span = cs % n_spans; cs /= n_spans;
+    const int h = cs % g.H; cs /= g.H;
+    const int blk = cs % g.nblk; cs /= g.nblk;
+    const int kvi = cs;
+    const int t_first = tok_begin + range * kItemTokens;
+    const int t_last = min(tok_begin + n_tok, t_first + kItemTokens);
+    const int n_tiles = (t_last - t_first + kTileTokens - 1) / kTileTokens;
+
+    // all MMAs of the previous item have completed (each set waited for its commits)
+    __syncthreads();
+    // prefetch the first two raw tiles of this item
+    if (tid == 0) {
+      for (int tl = 0; tl < min(2, n_tiles); ++tl) {
+        const int stg = (tile_counter + tl) % kRawStages;
+        const uint32_t bar = smem_addr(&bars[stg]);
+        mbar_expect_tx(bar, X::RAW);
+        tma_load_3d(smem_addr(raw + stg * X::RAW), &tmap, h * g.d + span * kSpan, t_first + tl * kTileTokens,
+                    kvi * g.T + blk * TC, bar);
+      }
+    }
+    // B tiles: [-2 C_k | n1 n2 n3 | 0] for the item's groups, K-major no-swizzle;
+    // nmax_s[gi] = max_k ||C_k||^2 (non-negative floats order like their bits)
+    if (tid < NGC) nmax_s[tid] = 0.f;
+    __syncthreads();
+    for (int e = tid; e < NGC * kEntries; e += kThreads) {
+      const int gi = e / kEntries, k = e % kEntries;
+      const int grp = span * NGC + gi;
+      const __nv_bfloat16* ce = cb + cb_off(g, layer, kvi, blk, h, grp) + (size_t)k * G;
+      unsigned char* bt = Bt + gi * X::B_TILE;
+      double n = 0.0;
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        const float v = __bfloat162float(ce[j]);
+        n += (double)v * (double)v;
+        *reinterpret_cast<__nv_bfloat16*>(bt + kmaj_off(k, j, SBO)) = __float2bfloat16_rn(-2.f * v);
+      }
+      const __nv_bfloat16 n1 = __double2bfloat16(n);
+      const double r1 = n - (double)__bfloat162float(n1);
+      const __nv_bfloat16 n2 = __double2bfloat16(r1);
+      const __nv_bfloat16 n3 = __double2bfloat16(r1 - (double)__bfloat162float(n2));
+      *reinterpret_cast<__nv_bfloat16*>(bt + kmaj_off(k, G, SBO)) = n1;
+      *reinterpret_cast<__nv_bfloat16*>(bt + kmaj_off(k, G + 1, SBO)) = n2;
+      *reinterpret_cast<__nv_bfloat16*>(bt + kmaj_off(k, G + 2, SBO)) = n3;
+      for (int j = G + 3; j < KP; ++j)
+        *reinterpret_cast<__nv_bfloat16*>(bt + kmaj_off(k, j, SBO)) = __float2bfloat16_rn(0.f);
+      atomicMax(reinterpret_cast<int*>(&nmax_s[gi]), __float_as_int((float)n));
+    }
+    fence_proxy_async();
+    __syncthreads();
+
+    for (int tl = 0; tl < n_tiles && !failed; ++tl, ++tile_counter) {
+      const int stg = tile_counter % kRawStages;
+      const int t0 = t_first + tl * kTileTokens;
+      if (__syncthreads_or(!mbar_wait(smem_addr(&bars[stg]), raw_phase[stg], kWaitIters))) {
+        failed = true;
+        break;
+      }
+      raw_phase[stg] ^= 1u;
+      const unsigned char* rw = raw + stg * X::RAW;
+      const bool valid_row = t0 + row < t_last;
+
+      // each set handles groups gi = set, set + 2, ...
+      for (int gi = set; gi < NGC; gi += 2) {
+        // A row: joint vector of token t0+row, group gi: element s*c+e = raw[s][row][gi*c+e]
+        unsigned char* at = At + gi * X::A_TILE;
+        float xx = 0.f;
+        __nv_bfloat16 xv[G];
+#pragma unroll
+        for (int s2 = 0; s2 < TC; ++s2)
+#pragma unroll
+          for (int e = 0; e < C; ++e) {
+            const __nv_bfloat16 v =
+                *reinterpret_cast<const __nv_bfloat16*>(rw + ((s2 * kTileTokens + row) * kSpan + gi * C + e) * 2);
+            xv[s2 * C + e] = v;
+            const float f = __bfloat162float(v);
+            xx = fmaf(f, f, xx);
+          }
+#pragma unroll
+        for (int k8 = 0; k8 < G / 8; ++k8) {
+          uint4 w;
+          uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            wp[q] = (uint32_t)__bfloat16_as_ushort(xv[k8 * 8 + 2 * q]) |
+                    ((uint32_t)__bfloat16_as_ushort(xv[k8 * 8 + 2 * q + 1]) << 16);
+          *reinterpret_cast<uint4*>(at + kmaj_off(row, k8 * 8, SBO)) = w;
+        }
+        {
+          const uint32_t one = 0x3f80u;   // bf16 1.0
+          uint4 w = make_uint4(one | (one << 16), one, 0u, 0u);
+          *reinterpret_cast<uint4*>(at + kmaj_off(row, G, SBO)) = w;
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        named_sync(1 + set, kRows);
+        if (row == 0) {
+          tc_fence_after();
+          const uint32_t a0 = smem_addr(at), b0 = smem_addr(Bt + gi * X::B_TILE);
+#pragma unroll
+          for (int ks = 0; ks < X::KSTEPS; ++ks)
+            mma_bf16(tmem_set, smem_desc(a0 + ks * 256, SBO), smem_desc(b0 + ks * 256, SBO), kIdesc, ks > 0);
+          mma_commit(smem_addr(&bars[kRawStages + set]));
+        }
+        if (!mbar_wait(smem_addr(&bars[kRawStages + set]), mma_phase, kWaitIters)) fail_s[set] = 1;
+        tc_fence_after();
+        named_sync(1 + set, kRows);
+        const bool ok = fail_s[set] == 0;      // uniform over the set
+
+        // epilogue: min of row, then the candidates within eps of it
+        const float eps = ldexpf(xx + nmax_s[gi], -14);
+        float m0 = INFINITY, m1 = INFINITY, m2 = INFINITY, m3 = INFINITY;
+#pragma unroll 1
+        for (int q = 0; q < kEntries / 32; ++q) {
+          float v[32];
+          tmem_ld32(tmem_set + lane_addr + q * 32, v);
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            m0 = fmin3(m0, v[i], v[i + 1]);
+            m1 = fmin3(m1, v[i + 2], v[i + 3]);
+            m2 = fmin3(m2, v[i + 4], v[i + 5]);
+            m3 = fmin3(m3, v[i + 6], v[i + 7]);
+          }
+        }
+        const float thr = fminf(fminf(m0, m1), fminf(m2, m3)) + eps;
+        uint32_t cand = 0;                 // (k+1) of every candidate, 9 bits each, last in the low bits
+#pragma unroll 1
+        for (int q = 0; q < kEntries / 32; ++q) {
+          float v[32];
+          tmem_ld32(tmem_set + lane_addr + q * 32, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (v[i] <= thr) cand = (cand << 9) + (uint32_t)(q * 32 + i + 1);
+        }
+        int code = (int)cand - 1;
+        const bool tie = cand >= 512u;
+        if (__any_sync(0xffffffffu, tie && valid_row)) {
+          // near-tie: exact fp64 direct-form distances of the candidates
+          double best = 1e300;
+          int bk = 0;
+#pragma unroll 1
+          for (int q = 0; q < kEntries / 32; ++q) {
+            float v[32];
+            tmem_ld32(tmem_set + lane_addr + q * 32, v);
+            if (tie) {
+              for (int i = 0; i < 32; ++i) {
+                if (v[i] <= thr) {
+                  const int k = q * 32 + i;
+                  const unsigned char* bt = Bt + gi * X::B_TILE;
+                  double d2 = 0.0;
+                  for (int j = 0; j < G; ++j) {
+                    const double cj =
+                        -0.5 * (double)__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(bt + kmaj_off(k, j, SBO)));
+                    const double df = (double)__bfloat162float(xv[j]) - cj;
+                    d2 = fma(df, df, d2);
+                  }
+                  if (d2 < best) { best = d2; bk = k; }
+                }
+              }
+            }
+          }
+          if (tie) code = bk;
+        }
+        tc_fence_before();
+        if (valid_row && ok) {
+          const int cn = coded_offset + (t0 + row - tok_begin);
+          uint8_t* page = idx + idx_page_off(g, layer, blk, req, h, cn >> 3);
+          page[kvi * g.ng * kPage + (span * NGC + gi) * kPage + (cn & 7)] = (uint8_t)code;
+        }
+        named_sync(1 + set, kRows);     // the set's TMEM columns and A tile are free again
+        mma_phase ^= 1u;                // one completed phase of this set's barrier per group
+        if (!ok) break;
+      }
+      if (__syncthreads_or(fail_s[0] | fail_s[1])) failed = true;
+      // refill this raw stage with the tile two ahead
+      if (tid == 0 && tl + 2 < n_tiles) {
+        const uint32_t bar = smem_addr(&bars[stg]);
+        mbar_expect_tx(bar, X::RAW);
+        tma_load_3d(smem_addr(raw + stg * X::RAW), &tmap, h * g.d + span * kSpan, t0 + 2 * kTileTokens,
+                    kvi * g.T + blk * TC, bar);
+      }
+    }
+  }
+  if (failed && tid == 0) set_status(st, LVQ_ETIMEOUT);
+  if (failed && row == 0)   // a set whose MMA wait gave up lets it finish before TMEM is freed
+    mbar_wait(smem_addr(&bars[kRawStages + set]), mma_phase, kWaitIters);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" :: "r"(tmem_base) : "memory");
+}
+
+}  // namespace tc
+
+bool encode_tc_supported(int G, int c) { return (G == 16 || G == 32) && (c == 4 || c == 8) && c < G; }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda dependency)
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+template <int G, int C>
+static cudaError_t encode_tc_as(const Geo& g, int layer, int req, const __nv_bfloat16* kv, int64_t tok_stride,
+                                int kv_tokens, int tok_begin, int n_tok, int coded_offset,
+                                const __nv_bfloat16* cb, uint8_t* idx, int32_t* st, cudaStream_t s) {
+  using X = tc::Enc<G, C>;
+  auto enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap map;
+  // dims: channels of a token row (H*d), tokens, (kv, step) planes
+  cuuint64_t dims[3] = {(cuuint64_t)g.H * g.d, (cuuint64_t)kv_tokens, (cuuint64_t)2 * g.T};
+  cuuint64_t strides[2] = {(cuuint64_t)tok_stride * 2, (cuuint64_t)tok_stride * kv_tokens * 2};
+  cuuint32_t box[3] = {tc::kSpan, tc::kTileTokens, (cuuint32_t)X::TC};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16*>(kv), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+
+  static bool attr_set[kMaxDevices] = {};
+  static int n_sm[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    e = cudaFuncSetAttribute(tc::encode_tc_kernel<G, C>, cudaFuncAttributeMaxDynamicSharedMemorySize, X::SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&n_sm[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const long n_sets = 2L * g.nblk * g.H * (g.d / tc::kSpan);
+  const long items = n_sets * ((n_tok + tc::kItemTokens - 1) / tc::kItemTokens);
+  const int grid = (int)std::min<long>(items, n_sm[dev]);
+  tc::encode_tc_kernel<G, C><<<grid, tc::kThreads, X::SMEM, s>>>(map, g, layer, req, tok_begin, n_tok,
+                                                                  coded_offset, cb, idx, st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_encode_tc(const Geo& g, int layer, int req, const __nv_bfloat16* kv, int64_t tok_stride,
+                             int kv_tokens, int tok_begin, int n_tok, int coded_offset,
+                             const __nv_bfloat16* cb, uint8_t* idx, int32_t* st, cudaStream_t s) {
+  if (n_tok == 0) return cudaSuccess;
+#define LVQ_ETC(GG, CC)                                                                                  \
+  if (g.G == GG && g.c == CC)                                                                            \
+    return encode_tc_as<GG, CC>(g, layer, req, kv, tok_stride, kv_tokens, tok_begin, n_tok, coded_offset, \
+                                cb, idx, st, s);
+  LVQ_ETC(16, 4) LVQ_ETC(16, 8) LVQ_ETC(32, 4) LVQ_ETC(32, 8)
+#undef LVQ_ETC
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace lvq

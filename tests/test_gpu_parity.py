@@ -43,10 +43,16 @@ def check_codes(gpu_codes: np.ndarray, X: np.ndarray, cb: np.ndarray):
 
 # ----------------------------------------------------------------------------------- encode
 
-@pytest.mark.parametrize("name,ntok,offset", [("tiny", 492, 0), ("ouro14_g16_32k", 333, 5),
-                                              ("ouro14_g32_b32", 130, 8), ("ouro14_tc2_64k", 77, 3)])
-def test_encode_prefill_matches_oracle(name, ntok, offset):
-    w = _reduced(name, n_layers=1) if name != "tiny" else synth.WORKLOADS[name]
+@pytest.mark.parametrize("name,ntok,offset,extra", [
+    ("tiny", 492, 0, {}),
+    ("ouro14_g16_32k", 333, 5, {}),
+    ("ouro14_g16_32k", 2100, 0, {"n_kv_heads": 2, "n_q_heads": 2}),     # several token tiles and items
+    ("ouro14_g32_b32", 130, 8, {}),
+    ("ouro14_tc2_64k", 77, 3, {}),
+    ("ouro14_g16_32k", 200, 1, {"Tc": 1, "n_kv_heads": 2, "n_q_heads": 2}),   # c = 16: fp64 direct form
+])
+def test_encode_prefill_matches_oracle(name, ntok, offset, extra):
+    w = _reduced(name, n_layers=1, **extra) if name != "tiny" else synth.WORKLOADS[name]
     case = Hl.build_case(w, layers=1, ctx=[w.n_sink + ntok + offset + w.n_recent], coded=[ntok + offset],
                          codes_from="none")
     c = case.cache
