@@ -203,6 +203,24 @@ def build_cache(w, lvq, synth, torch, extra_tokens: int, device, request_seed: i
     return cfg, cache
 
 
+def reduce_max(value: float, device) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_plan(rank: int, world: int, batch_per_rank: int) -> dict:
+    """Weak scaling by request: rank r serves requests [r*B, (r+1)*B) with its own seeds;
+    no data crosses ranks."""
+    return {"first_request": rank * batch_per_rank, "requests": batch_per_rank,
+            "seed": rank, "global_batch": world * batch_per_rank}
+
+
 def choose_splits(w, n_sm: int) -> int:
     # one CTA per SM: (splits + 1 bf16 CTA) * heads * requests <= SMs
     return max(1, min(128, n_sm // (w.batch * w.n_q_heads) - 1))
@@ -255,7 +273,8 @@ def gpu_arm(args):
         return
     w = synth.WORKLOADS[WORKLOAD]
     replays = 2 * args.steps + args.warmup + 3          # every graph replay adds 8 tokens
-    cfg, cache = build_cache(w, lvq, synth, torch, TOKENS_PER_STEP * (replays + 4), device, rank)
+    cfg, cache = build_cache(w, lvq, synth, torch, TOKENS_PER_STEP * (replays + 4), device,
+                             replica_plan(rank, world, w.batch)["seed"])
     lay = cache.lay
     n_sm = torch.cuda.get_device_properties(device).multi_processor_count
     ns = args.splits or choose_splits(w, n_sm)
@@ -319,13 +338,10 @@ def gpu_arm(args):
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-    ms = t_start.elapsed_time(t_end)
+    ms = reduce_max(t_start.elapsed_time(t_end), device)
     cache.check_status("timed")
-    if world > 1:
-        tt = torch.tensor([ms], device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
-    tokens = TOKENS_PER_STEP * args.steps * B * world
+    plan = replica_plan(rank, world, B)
+    tokens = TOKENS_PER_STEP * args.steps * plan["global_batch"]
     value = tokens / (ms / 1e3)
 
     # ---- decode kernel timing: a graph of the 96 attentions of one token, event-timed
@@ -374,11 +390,7 @@ def gpu_arm(args):
             out_host.copy_(out_all, non_blocking=True)
         t1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = reduce_max(t0.elapsed_time(t1), device)
     e2e_value = tokens / (e2e_ms / 1e3)
     cache.check_status("e2e")
 
