@@ -107,60 +107,125 @@ __device__ inline int page_due(const Geo& g, int ctx, int coded) {
   return 1;
 }
 
-// One warp per codebook (layer, kv, blk, h, grp) and request; lane l scans
-// entries l, l+32, ..., then the warp takes the lexicographic (distance, k)
-// minimum, which is the lowest index among equal distances.
-constexpr int kPageWarps = 4;
+// One CTA per codebook (layer, kv, blk, h, grp), looping over the requests whose
+// page is due, so each codebook is read from memory once.  The codebook and
+// its squared norms sit in shared memory; warp t takes token t of the page and
+// lane l the entries l, l + 32, ...  Distances are first taken in the fp32
+// expansion form n_k - 2 x.C_k; every entry within
+// eps = 2^-14 (||x||^2 + max_k n_k) of the minimum is a candidate (the fp32
+// error is far below eps), and when there are several the candidates are
+// rescored exactly in the fp64 direct form, lowest index on ties.
+constexpr int kPageThreads = 32 * kPage;
 
-__global__ void __launch_bounds__(32 * kPageWarps) encode_page_kernel(
-    Geo g, const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ coded_len,
-    const __nv_bfloat16* __restrict__ ring, const __nv_bfloat16* __restrict__ cb,
-    uint8_t* __restrict__ idx, int32_t* st) {
-  const int b = blockIdx.y;
-  const int lane = threadIdx.x & 31;
-  long cid = (long)blockIdx.x * kPageWarps + (threadIdx.x >> 5);
-  const long n_cb = (long)g.L * 2 * g.nblk * g.H * g.ng;
-  if (cid >= n_cb) return;
-  const int ctx = ctx_len[b], coded = coded_len[b];
-  const int due = page_due(g, ctx, coded);
-  if (due < 0) { if (cid == 0 && lane == 0) set_status(st, LVQ_ECAPACITY); return; }
-  if (due == 0) return;
-
+template <int G, int C>
+__global__ void __launch_bounds__(kPageThreads, 2) encode_page_kernel(
+    Geo g, int batch, const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ coded_len,
+    const __nv_bfloat16* __restrict__ ring, const __nv_bfloat16* __restrict__ cb, uint8_t* __restrict__ idx,
+    int32_t* st) {
+  constexpr int TC = G / C;
+  __shared__ float cbs[kEntries * G];     // fp32 copies of the bf16 entries (exact)
+  __shared__ float nrm[kEntries];
+  __shared__ float nmax_s;
+  long cid = blockIdx.x;
   const int grp = (int)(cid % g.ng); cid /= g.ng;
   const int h = (int)(cid % g.H); cid /= g.H;
   const int blk = (int)(cid % g.nblk); cid /= g.nblk;
   const int kvi = (int)(cid % 2); cid /= 2;
   const int layer = (int)cid;
+  const int tid = threadIdx.x, lane = tid & 31, t = tid >> 5;
 
-  // this lane's 8 entries, widened to fp64
-  const __nv_bfloat16* C = cb + cb_off(g, layer, kvi, blk, h, grp);
-  uint8_t* page_base = idx + idx_page_off(g, layer, blk, b, h, 0) + kvi * g.ng * kPage + grp * kPage;
-  for (int t = 0; t < kPage; ++t) {
-    const int cn = coded + t;
-    const int slot = cn % g.R;           // position S + cn lives in slot (cn mod R)
-    double x[32];
-    for (int s = 0; s < g.Tc; ++s) {
-      const __nv_bfloat16* p = ring + ring_off(g, layer, kvi, blk * g.Tc + s, b, h, slot) + grp * g.c;
-      for (int e = 0; e < g.c; ++e) x[s * g.c + e] = (double)__bfloat162float(p[e]);
+  bool any = false;
+  for (int b = 0; b < batch; ++b) any |= page_due(g, ctx_len[b], coded_len[b]) == 1;
+  if (!any) return;
+
+  const __nv_bfloat16* Cg = cb + cb_off(g, layer, kvi, blk, h, grp);
+  for (int i = tid; i < kEntries * G; i += kPageThreads) cbs[i] = __bfloat162float(Cg[i]);
+  if (tid == 0) nmax_s = 0.f;
+  __syncthreads();
+  {
+    const int k = tid;                    // kPageThreads == kEntries
+    double n = 0.0;
+#pragma unroll
+    for (int j = 0; j < G; ++j) n += (double)cbs[k * G + j] * (double)cbs[k * G + j];
+    nrm[k] = (float)n;
+    atomicMax(reinterpret_cast<int*>(&nmax_s), __float_as_int((float)n));
+  }
+  __syncthreads();
+
+  for (int b = 0; b < batch; ++b) {
+    const int ctx = ctx_len[b], coded = coded_len[b];
+    const int due = page_due(g, ctx, coded);
+    if (due < 0) {
+      if (blockIdx.x == 0 && tid == 0) set_status(st, LVQ_ECAPACITY);
+      continue;
     }
-    double best = 1e300;
-    int bk = 0;
-    for (int i = 0; i < kEntries / 32; ++i) {
-      const int k = lane + 32 * i;
-      const __nv_bfloat16* ce = C + (size_t)k * g.G;
-      double acc = 0.0;
-      for (int j = 0; j < g.G; ++j) {
-        double df = x[j] - (double)__bfloat162float(ce[j]);
-        acc = fma(df, df, acc);
+    if (due == 0) continue;
+    const int cn = coded + t;             // this warp's token, coded slot cn
+    const int slot = cn % g.R;            // position S + cn lives in slot (cn mod R)
+    float x[G];
+    float xx = 0.f;
+#pragma unroll
+    for (int s2 = 0; s2 < TC; ++s2) {
+      const __nv_bfloat16* p = ring + ring_off(g, layer, kvi, blk * TC + s2, b, h, slot) + grp * C;
+#pragma unroll
+      for (int e = 0; e < C; ++e) {
+        x[s2 * C + e] = __bfloat162float(p[e]);
+        xx = fmaf(x[s2 * C + e], x[s2 * C + e], xx);
       }
-      if (acc < best) { best = acc; bk = k; }
     }
-    for (int off = 16; off > 0; off >>= 1) {
-      double ob = __shfl_xor_sync(0xffffffffu, best, off);
-      int ok = __shfl_xor_sync(0xffffffffu, bk, off);
-      if (ob < best || (ob == best && ok < bk)) { best = ob; bk = ok; }
+    float dv[kEntries / 32];
+    float best = INFINITY;
+#pragma unroll
+    for (int i = 0; i < kEntries / 32; ++i) {
+      const float* ce = cbs + (lane + 32 * i) * G;
+      float dot = 0.f;
+#pragma unroll
+      for (int j = 0; j < G; ++j) dot = fmaf(x[j], ce[j], dot);
+      dv[i] = fmaf(-2.f, dot, nrm[lane + 32 * i]);
+      best = fminf(best, dv[i]);
     }
-    if (lane == 0) page_base[(size_t)(cn >> 3) * g.page_bytes + (cn & 7)] = (uint8_t)bk;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) best = fminf(best, __shfl_xor_sync(0xffffffffu, best, o));
+    const float thr = best + ldexpf(xx + nmax_s, -14);
+    int n_cand = 0, k_cand = kEntries;
+#pragma unroll
+    for (int i = 0; i < kEntries / 32; ++i)
+      if (dv[i] <= thr) { ++n_cand; k_cand = min(k_cand, lane + 32 * i); }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      n_cand += __shfl_xor_sync(0xffffffffu, n_cand, o);
+      k_cand = min(k_cand, __shfl_xor_sync(0xffffffffu, k_cand, o));
+    }
+    int code = k_cand;
+    if (n_cand > 1) {
+      // near-tie: exact fp64 direct-form distances of the candidates, lowest index on ties
+      double bd = 1e300;
+      int bk = kEntries;
+#pragma unroll 1
+      for (int i = 0; i < kEntries / 32; ++i) {
+        if (dv[i] <= thr) {
+          const int k = lane + 32 * i;
+          double acc = 0.0;
+#pragma unroll
+          for (int j = 0; j < G; ++j) {
+            const double df = (double)x[j] - (double)cbs[k * G + j];
+            acc = fma(df, df, acc);
+          }
+          if (acc < bd) { bd = acc; bk = k; }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double ob = __shfl_xor_sync(0xffffffffu, bd, o);
+        const int ok = __shfl_xor_sync(0xffffffffu, bk, o);
+        if (ob < bd || (ob == bd && ok < bk)) { bd = ob; bk = ok; }
+      }
+      code = bk;
+    }
+    if (lane == 0) {
+      uint8_t* page = idx + idx_page_off(g, layer, blk, b, h, cn >> 3);
+      page[kvi * g.ng * kPage + grp * kPage + (cn & 7)] = (uint8_t)code;
+    }
   }
 }
 
@@ -171,14 +236,24 @@ __global__ void advance_kernel(Geo g, int batch, const int32_t* __restrict__ ctx
   }
 }
 
+template <int G, int C>
+static cudaError_t encode_page_as(const Geo& g, int batch, const int32_t* ctx_len, int32_t* coded_len,
+                                  const __nv_bfloat16* ring, const __nv_bfloat16* cb, uint8_t* idx, int32_t* st,
+                                  cudaStream_t s) {
+  const long n_cb = (long)g.L * 2 * g.nblk * g.H * g.ng;
+  encode_page_kernel<G, C><<<(unsigned)n_cb, kPageThreads, 0, s>>>(g, batch, ctx_len, coded_len, ring, cb, idx, st);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_encode_page(const Geo& g, int batch, const int32_t* ctx_len, int32_t* coded_len,
                                const __nv_bfloat16* ring, const __nv_bfloat16* cb, uint8_t* idx,
                                int32_t* st, cudaStream_t s) {
   if (batch == 0) return cudaSuccess;
-  const long n_cb = (long)g.L * 2 * g.nblk * g.H * g.ng;
-  dim3 grid((unsigned)((n_cb + kPageWarps - 1) / kPageWarps), batch);
-  encode_page_kernel<<<grid, 32 * kPageWarps, 0, s>>>(g, ctx_len, coded_len, ring, cb, idx, st);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = cudaErrorInvalidValue;
+#define LVQ_PG(GG, CC) \
+  if (g.G == GG && g.c == CC) e = encode_page_as<GG, CC>(g, batch, ctx_len, coded_len, ring, cb, idx, st, s);
+  LVQ_PG(16, 4) LVQ_PG(16, 8) LVQ_PG(16, 16) LVQ_PG(32, 4) LVQ_PG(32, 8) LVQ_PG(32, 16)
+#undef LVQ_PG
   if (e != cudaSuccess) return e;
   advance_kernel<<<1, 256, 0, s>>>(g, batch, ctx_len, coded_len);
   return cudaGetLastError();

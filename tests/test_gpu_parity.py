@@ -251,3 +251,28 @@ def test_page_encode_matches_oracle_and_advances():
     b4 = before.view(c.idx_view().shape)
     assert torch.equal(after[:, :, 1], b4[:, :, 1])
     assert torch.equal(after[:, :, 0, :, :12], b4[:, :, 0, :, :12])
+
+
+def test_decode_guard_fallback_large_scores():
+    """Keys of one entry are scaled by 100 and used only outside each warp's first page: later
+    scores exceed the split's reference maximum by far more than 2^64, which forces the exact
+    recomputation path.  The result must still match the oracle."""
+    w = synth.WORKLOADS["tiny"]
+    case = Hl.build_case(w, layers=1, ctx=[512])
+    c = case.cache
+    cbv = c.cb_view()
+    cbv[0, 0, :, :, :, 7, :] = (cbv[0, 0, :, :, :, 7, :].float() * 100).to(torch.bfloat16)
+    case.cb[0][0, :, :, :, 7, :] = cbv[0, 0, :, :, :, 7, :].cpu()
+    lvq.lvq_pack_codebooks(case.cfg, c.lay, c.cb, c.cbp)
+    ck, cv = case.codes[(0, 0)]
+    ck = ck.clone()
+    n = torch.arange(ck.shape[1])
+    first_pages = ((n // 8) % 4) == 0          # the first page of every warp's 4-page run
+    sel = ck[:, first_pages]
+    sel[sel == 7] = 8
+    ck[:, first_pages] = sel
+    Hl.put_codes(c, 0, 0, 0, ck.cuda())
+    case.codes[(0, 0)] = (ck, cv)
+    for step in range(w.T):
+        q = synth.queries(w, 0, step).cuda()
+        _check_decode(case, 0, step, q, 1)
