@@ -223,6 +223,32 @@ LVQ_API lvq_status lvq_dequantize(const lvq_config* cfg, const lvq_layout* lay, 
                           const void* cbp, int32_t tok_begin, int32_t n_tok, void* out,
                           void* stream);
 
+/* Decode attention without a caller-supplied workspace.  The pages have no
+ * counterpart of this entry point: it exists for callers that cannot allocate
+ * device memory for the workspace -- for example a plugin inside a serving
+ * engine whose memory pool owns the whole device, or a deployment that forbids
+ * allocations once it has reserved its memory budget.
+ *
+ * Arguments and results are those of lvq_decode_attention without
+ * `workspace`.  The workspace is a file-scope device array inside the library
+ * (4 MiB, held by every GPU that loads the library until the process exits):
+ *   - a layout whose workspace_bytes exceeds 4 MiB is rejected with
+ *     LVQ_ECAPACITY before anything is launched;
+ *   - the call allocates nothing (no cudaMalloc or allocating library
+ *     routine); it zeroes the merge counters with cudaMemsetAsync on `stream`;
+ *   - the first call on a device looks up the array's device address with that
+ *     device current; make that first call before any stream capture;
+ *   - every call shares the one array: calls that overlap on the GPU (other
+ *     streams, other host threads, other decode calls in flight) race and must
+ *     be serialized by the caller. */
+LVQ_API lvq_status lvq_decode_attention_noalloc(const lvq_config* cfg, const lvq_layout* lay, int32_t layer,
+                                                int32_t step, int32_t batch, const void* q,
+                                                const int32_t* ctx_len, const int32_t* coded_len,
+                                                const void* sink, const void* ring, const uint8_t* idx,
+                                                const void* cbp, const float* rope, int32_t num_splits,
+                                                float* out, float* lse, float* split_lse,
+                                                int32_t* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -233,3 +233,74 @@ lvq_status lvq_dequantize(const lvq_config* cfg, const lvq_layout* lay, int32_t 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------- allocation-free decode
+//
+// Some callers cannot allocate device memory for the decode workspace: for
+// example a plugin running inside a serving engine whose memory pool owns the
+// whole device, or a deployment that fixes its memory budget at start-up and
+// forbids allocations afterwards.  For them lvq_decode_attention_noalloc uses
+// a workspace that lives in the library itself: the file-scope device array
+// below, which every GPU that loads the library holds until the process exits.
+
+namespace {
+
+constexpr size_t kNoallocWorkspaceBytes = size_t(4) << 20;   // the stated maximum: 4 MiB
+static __device__ __align__(256) float g_noalloc_workspace[kNoallocWorkspaceBytes / sizeof(float)];
+
+// Device address of g_noalloc_workspace, looked up once per device with that
+// device current.  In host code the array's name is only a stand-in, never a
+// device address.
+float* noalloc_workspace(int dev) {
+  static float* addr[kMaxDevices] = {};
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_workspace) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<float*>(p);
+  }
+  return addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+lvq_status lvq_decode_attention_noalloc(const lvq_config* cfg, const lvq_layout* lay, int32_t layer, int32_t step,
+                                        int32_t batch, const void* q, const int32_t* ctx_len,
+                                        const int32_t* coded_len, const void* sink, const void* ring,
+                                        const uint8_t* idx, const void* cbp, const float* rope, int32_t num_splits,
+                                        float* out, float* lse, float* split_lse, int32_t* dev_status,
+                                        void* stream) {
+  Geo g;
+  lvq_status s = check_all(cfg, lay, &g);
+  if (s != LVQ_OK) return s;
+  if (lay->workspace_bytes > kNoallocWorkspaceBytes) return LVQ_ECAPACITY;
+  if (layer < 0 || layer >= g.L || step < 0 || step >= g.T || batch < 0 || batch > g.B || num_splits < 1 ||
+      num_splits > g.max_splits)
+    return LVQ_EINVAL;
+  if (batch > 0) {
+    const void* ptrs[] = {q, sink, ring, idx, cbp, rope, out, lse};
+    for (const void* p : ptrs)
+      if (!p || !aligned16(p)) return LVQ_EINVAL;
+    if (!ctx_len || !coded_len || (split_lse && ((uintptr_t)split_lse & 3u))) return LVQ_EINVAL;
+  }
+  if ((s = check_device()) != LVQ_OK) return s;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LVQ_ECUDA;
+  float* ws = noalloc_workspace(dev);
+  if (!ws) return LVQ_ECUDA;
+  if (batch == 0) return LVQ_OK;
+  // the merge counters after the partials must start at zero (a previous call that
+  // failed part-way could have left some set); the partials need no clearing
+  const size_t partial_floats = (size_t)g.B * g.Hq * (g.max_splits + 1) * (g.d + 2);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws + partial_floats, 0, (size_t)g.B * g.Hq * sizeof(int32_t), st) != cudaSuccess)
+    return LVQ_ECUDA;
+  return cuda_status(launch_decode(g, layer, step, batch, static_cast<const __nv_bfloat16*>(q), ctx_len, coded_len,
+                                   static_cast<const __nv_bfloat16*>(sink), static_cast<const __nv_bfloat16*>(ring),
+                                   idx, static_cast<const __nv_bfloat16*>(cbp), rope, num_splits, ws, out, lse,
+                                   split_lse, dev_status, st));
+}
+
+}  // extern "C"

@@ -58,6 +58,8 @@ _SIGS = {
     "lvq_dequantize": [ctypes.POINTER(lvq_config), ctypes.POINTER(lvq_layout), _I32, _I32, _I32, _I32, _P,
                        _P, _I32, _I32, _P, _P],
     "lvq_status_string": [_I32],
+    "lvq_decode_attention_noalloc": [ctypes.POINTER(lvq_config), ctypes.POINTER(lvq_layout), _I32, _I32, _I32,
+                                     _P, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P, _P],
 }
 EXPORTED = tuple(_SIGS)
 
@@ -173,6 +175,23 @@ def lvq_decode_attention(cfg, lay, layer, step, batch, q, ctx_len, coded_len, si
         _ptr(lse, "lse", torch.float32, 4 * batch * cfg.n_q_heads),
         _ptr(split_lse, "split_lse", torch.float32, 4 * batch * cfg.n_q_heads * (num_splits + 1), optional=True),
         _ptr(dev_status, "dev_status", torch.int32, 4), _stream(stream)), "lvq_decode_attention")
+
+
+def lvq_decode_attention_noalloc(cfg, lay, layer, step, batch, q, ctx_len, coded_len, sink, ring, idx, cbp, rope,
+                                 num_splits, out, lse, dev_status, split_lse=None, stream=None):
+    """lvq_decode_attention with the library's own 4 MiB device workspace (no workspace argument)."""
+    d = cfg.head_dim
+    _check(lib().lvq_decode_attention_noalloc(
+        ctypes.byref(cfg), ctypes.byref(lay), layer, step, batch,
+        _ptr(q, "q", torch.bfloat16, 2 * batch * cfg.n_q_heads * d),
+        _ptr(ctx_len, "ctx_len", torch.int32, 4 * batch), _ptr(coded_len, "coded_len", torch.int32, 4 * batch),
+        _ptr(sink, "sink", torch.bfloat16, lay.sink_bytes), _ptr(ring, "ring", torch.bfloat16, lay.ring_bytes),
+        _ptr(idx, "idx", torch.uint8, lay.idx_bytes), _ptr(cbp, "cbp", torch.bfloat16, lay.cbp_bytes),
+        _ptr(rope, "rope", torch.float32, lay.rope_bytes), num_splits,
+        _ptr(out, "out", torch.float32, 4 * batch * cfg.n_q_heads * d),
+        _ptr(lse, "lse", torch.float32, 4 * batch * cfg.n_q_heads),
+        _ptr(split_lse, "split_lse", torch.float32, 4 * batch * cfg.n_q_heads * (num_splits + 1), optional=True),
+        _ptr(dev_status, "dev_status", torch.int32, 4), _stream(stream)), "lvq_decode_attention_noalloc")
 
 
 def lvq_dequantize(cfg, lay, layer, step, req, kv, idx, cbp, tok_begin, n_tok, out, stream=None):
