@@ -222,8 +222,8 @@ def replica_plan(rank: int, world: int, batch_per_rank: int) -> dict:
 
 
 def choose_splits(w, n_sm: int) -> int:
-    # one CTA per SM: (splits + 1 bf16 CTA) * heads * requests <= SMs
-    return max(1, min(128, n_sm // (w.batch * w.n_q_heads) - 1))
+    # one CTA per SM: splits * heads * requests <= SMs
+    return max(1, min(128, n_sm // (w.batch * w.n_q_heads)))
 
 
 def decode_bytes_per_launch(w, lay, coded: int, recent: int) -> int:

@@ -98,12 +98,13 @@ typedef struct {
   int32_t n_blocks;     /* n_blk = T / Tc: index rows per token, head and K/V */
   int32_t ring_tokens;  /* R = n_recent + page_tokens: recent-window slots */
   int32_t max_pages;    /* coded pages per (layer, block, request, head) */
-  int32_t page_bytes;   /* bytes of one coded page: 2 * n_g * 8 (K then V) */
+  int32_t page_bytes;   /* bytes of one coded page of K or of V: n_g * 8 */
   int32_t rope_coarse;  /* rows of the coarse RoPE table (positions 8k) */
   int32_t reserved;
-  /* uint8 codes, [layer][n_blk][B][Hkv][page][kv][n_g][8]: byte (g, j) of a
+  /* uint8 codes, [layer][n_blk][B][Hkv][kv][page][n_g][8]: byte (g, j) of a
    * page holds group g's code of the page's token j (token n of the coded
-   * region sits in page n/8 at j = n%8). */
+   * region sits in page n/8 at j = n%8).  The K pages of a (layer, block,
+   * request, head) form one contiguous stream, followed by its V pages. */
   size_t idx_bytes;
   int64_t idx_strides[8];
   /* bf16 logical codebooks, [layer][kv][n_blk][Hkv][n_g][256][G]; element
@@ -127,9 +128,10 @@ typedef struct {
   /* fp32 RoPE tables: coarse [rope_coarse][d/2] (cos, sin) of 8k*theta_f,
    * then fine [8][d/2] (cos, sin) of r*theta_f.  Written by lvq_rope_table. */
   size_t rope_bytes;
-  /* scratch of lvq_decode_attention: fp32 split partials
-   * [B][Hq][max_splits + 1][d + 2], then int32 merge counters [B][Hq].  Zero
-   * it once before first use; every call leaves the counters at zero. */
+  /* scratch of lvq_decode_attention: fp32 partials
+   * [B][Hq][max_splits][2][d + 2] (per split: its coded tokens, its share of
+   * the bf16 tokens), then int32 merge counters [B][Hq].  Zero it once before
+   * first use; every call leaves the counters at zero. */
   size_t workspace_bytes;
 } lvq_layout;
 

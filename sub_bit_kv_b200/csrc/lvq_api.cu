@@ -39,7 +39,7 @@ Geo make_geo(const lvq_config* c) {
   g.P = max_coded > 0 ? (max_coded + kPage - 1) / kPage : 1;
   g.B = c->max_batch; g.max_ctx = c->max_ctx; g.max_splits = c->max_splits;
   g.RC = max((c->max_ctx + kPage - 1) / kPage, 64) + 16;   // rows cover offsets up to 512 positions
-  g.page_bytes = 2 * g.ng * kPage;
+  g.page_bytes = g.ng * kPage;
   return g;
 }
 
@@ -47,7 +47,7 @@ void fill_layout(const Geo& g, lvq_layout* o) {
   memset(o, 0, sizeof(*o));
   o->c = g.c; o->n_groups = g.ng; o->n_blocks = g.nblk; o->ring_tokens = g.R; o->max_pages = g.P;
   o->page_bytes = g.page_bytes; o->rope_coarse = g.RC;
-  const int64_t idims[8] = {g.L, g.nblk, g.B, g.H, g.P, 2, g.ng, kPage};
+  const int64_t idims[8] = {g.L, g.nblk, g.B, g.H, 2, g.P, g.ng, kPage};
   int64_t st = 1;
   for (int i = 7; i >= 0; --i) { o->idx_strides[i] = st; st *= idims[i]; }
   o->idx_bytes = (size_t)st;
@@ -69,7 +69,7 @@ void fill_layout(const Geo& g, lvq_layout* o) {
   for (int i = 6; i >= 0; --i) { o->ring_strides[i] = st; st *= rdims[i]; }
   o->ring_bytes = (size_t)st * 2;
   o->rope_bytes = (size_t)(g.RC + kPage) * (g.d / 2) * 2 * 4;
-  o->workspace_bytes = (size_t)g.B * g.Hq * (g.max_splits + 1) * (g.d + 2) * 4 + (size_t)g.B * g.Hq * 4;
+  o->workspace_bytes = ws_partial_floats(g) * 4 + (size_t)g.B * g.Hq * 4;
 }
 
 // Re-derives the layout and checks the caller's copy matches it.
@@ -293,7 +293,7 @@ lvq_status lvq_decode_attention_noalloc(const lvq_config* cfg, const lvq_layout*
   if (batch == 0) return LVQ_OK;
   // the merge counters after the partials must start at zero (a previous call that
   // failed part-way could have left some set); the partials need no clearing
-  const size_t partial_floats = (size_t)g.B * g.Hq * (g.max_splits + 1) * (g.d + 2);
+  const size_t partial_floats = ws_partial_floats(g);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(ws + partial_floats, 0, (size_t)g.B * g.Hq * sizeof(int32_t), st) != cudaSuccess)
     return LVQ_ECUDA;

@@ -19,9 +19,14 @@ struct Geo {
   int page_bytes;
 };
 
-__host__ __device__ inline size_t idx_page_off(const Geo& g, int layer, int blk, int b, int h, int page) {
-  return ((((size_t)layer * g.nblk + blk) * g.B + b) * g.H + h) * (size_t)g.P * g.page_bytes +
-         (size_t)page * g.page_bytes;
+// byte offset of the code stream [page][n_g][8] of (layer, blk, b, h, kv)
+__host__ __device__ inline size_t idx_stream_off(const Geo& g, int layer, int blk, int b, int h, int kv) {
+  return (((((size_t)layer * g.nblk + blk) * g.B + b) * g.H + h) * 2 + kv) * (size_t)g.P * g.page_bytes;
+}
+// byte offset of group grp's code of coded token n in that stream
+__host__ __device__ inline size_t idx_code_off(const Geo& g, int layer, int blk, int b, int h, int kv, int n,
+                                               int grp) {
+  return idx_stream_off(g, layer, blk, b, h, kv) + (size_t)(n >> 3) * g.page_bytes + grp * kPage + (n & 7);
 }
 // element offset of the packed step slice [256][ng][c] of (layer, kv, blk, h, s)
 __host__ __device__ inline size_t cbp_slice_off(const Geo& g, int layer, int kv, int blk, int h, int s) {
@@ -38,6 +43,12 @@ __host__ __device__ inline size_t sink_off(const Geo& g, int layer, int kv, int 
 // element offset of ring slot `slot` of (layer, kv, step, b, h)
 __host__ __device__ inline size_t ring_off(const Geo& g, int layer, int kv, int t, int b, int h, int slot) {
   return ((((((size_t)layer * 2 + kv) * g.T + t) * g.B + b) * g.H + h) * g.R + slot) * (size_t)g.d;
+}
+
+// fp32 partials of the decode workspace: [B][Hq][max_splits][coded, bf16][d + 2];
+// the int32 merge counters [B][Hq] follow them.
+__host__ __device__ inline size_t ws_partial_floats(const Geo& g) {
+  return (size_t)g.B * g.Hq * g.max_splits * 2 * (g.d + 2);
 }
 
 // Records the first device-side error: later errors do not overwrite it.

@@ -7,33 +7,43 @@
 // logsumexp.  Section "how it differs": keys are stored before RoPE and RoPE is
 // applied to the reconstructed key.
 //
-// Grid (num_splits + 1, query heads, requests); 15 compute warps and one
-// producer warp per CTA, one CTA per SM.
-//  * Coded split j < num_splits: the producer bulk-copies the step-t key and
-//    value slices of the head's codebooks ([256][n_g][c] bf16 each, one
-//    contiguous span each) and then the split's code pages, 480 tokens per
-//    chunk, through a 3-stage ring (cp.async.bulk into shared memory, no
-//    multicast; full/empty mbarriers).  Each compute warp takes 4 consecutive
-//    pages of every chunk.
-//  * Scores: lane (tq, P) of a compute warp owns pair-group P -- groups P and
-//    P + n_g/2, i.e. the RoPE frequencies f = P*c + e whose rotate-half
-//    partners are channels f and f + d/2 -- and every (32/n_p)-th token of the
-//    warp's pages.  With z_f = q'_f + i q'_{f+d/2} (the query rotated at its own
-//    position), a key k at position p scores
+// Grid (num_splits, query heads, requests); 15 compute warps and one producer
+// warp per CTA, one CTA per SM.  CTA j owns coded split j and every
+// num_splits-th bf16 token (sink and recent window), and writes two partials
+// (m, l, o): its coded split and its share of the bf16 tokens.
+//  * bf16 share: computed first, from global memory, while the step slices
+//    and the first code chunks are in flight.  One warp per token scores it
+//    against the query rotated to the token's position (the key's RoPE moved
+//    onto the query); 512 threads then sum the weighted value rows.
+//  * Coded split: the producer bulk-copies the step-t key slice ([256][n_g][c]
+//    bf16, one contiguous span), the value slice, and the split's code pages in
+//    480-token chunks through a 3-stage ring (cp.async.bulk, no multicast;
+//    full/empty mbarriers): the K pages of a super-chunk, then its V pages.
+//  * Phase A (scores): lane (tq, P) of a compute warp owns pair-group P --
+//    groups P and P + n_g/2, i.e. the RoPE frequencies f = P*c + e whose
+//    rotate-half partners are channels f and f + d/2 -- and every
+//    (32/n_p)-th token of the warp's pages.  With z_f = q'_f + i q'_{f+d/2}
+//    (the query rotated at its own position), a key k at position p scores
 //      sum_f Re(z_f e^{-i p theta_f}) k_f + Im(z_f e^{-i p theta_f}) k_{f+d/2}
 //    = q' . RoPE(k, p).  Along a lane's tokens (stride s) the factor
 //    W_n = z e^{-i p_n theta} obeys W_{n+1} = 2 cos(s theta) W_n - W_{n-1}: one
 //    packed f32x2 FMA per frequency for the rotation and one for the dot
 //    product; the recurrence is reseeded exactly at every chunk.  A code byte
-//    becomes its shared-memory row address in one byte permute.
-//  * Values: lane (tp, g) owns group g's c channels and accumulates
-//    p * V_slice[code][g] for every (32/n_g)-th token in fp32 registers, with
-//    an online softmax per warp (the warp's reference maximum is raised, and
-//    its accumulators rescaled, only when a score exceeds it by 2^16).
-//  * CTA num_splits computes the bf16 tokens' partial (sink and recent window)
-//    from shared-memory copies of the tokens and of the RoPE table rows.
-//  * The last CTA of a (request, head) to finish merges the partials by LSE
-//    (a counter in the workspace, returned to zero by that CTA).
+//    becomes its shared-memory row address in one byte permute.  Scores go to
+//    shared memory.
+//  * Between the phases: the exact maximum M of the super-chunk and
+//    S = sum 2^(s - M); every weight becomes the integer round(2^(s-M) * 2^k)
+//    with 2^k * S < 2^30, so that any sum of weights fits 31 bits and each
+//    weight is exact to 2^-31 of S.
+//  * Phase B (values): out = sum_t w_t V[code_t] = sum_(a, g) H[a][g] V[a][g],
+//    with H[a][g] the sum of the weights of the tokens whose group-g code is
+//    a.  Lane g adds its tokens' weights to H with 32-bit shared-memory
+//    atomics (integer adds: exact and order-independent; row a of H is 4*n_g
+//    bytes, so the 32 lanes of a warp hit 32 distinct banks).  One pass over
+//    the value slice then contracts H into o.
+//  * The last CTA of a (request, head) to finish merges the 2 * num_splits
+//    partials by LSE (a counter in the workspace, returned to zero by that
+//    CTA).
 #include "lvq_common.cuh"
 
 namespace lvq {
@@ -44,7 +54,9 @@ constexpr int kThr = kCT + 32;
 constexpr int kPPW = 4;                      // pages per warp per chunk
 constexpr int kChunk = kPage * kCW * kPPW;   // 480 coded tokens per chunk
 constexpr int kStages = 3;
-constexpr float kRaiseLog2 = 16.f;           // raise a warp's reference maximum beyond this margin
+constexpr int kSmemMax = 227 * 1024;
+constexpr int kBarCompute = 1;               // named barrier of the 15 compute warps
+constexpr int kMaxSuperChunks = 16;          // chunks per super-chunk, at most
 
 template <int D, int C>
 struct Dec {
@@ -54,24 +66,35 @@ struct Dec {
   static constexpr int TQ = 32 / NP;       // token phases of the score mapping
   static constexpr int TPL = kPage / TQ;   // score tokens per lane per page
   static constexpr int GRP = NP / TPL;     // lanes holding the same reduced score
-  static constexpr int TPV = 32 / NG;      // token phases of the value mapping
-  static constexpr int VPL = kPage / TPV;   // value tokens per lane per page
-  static constexpr int PAGE = 2 * NG * kPage;
+  static constexpr int TPV = 32 / NG;      // lanes per group in the value phase
+  static constexpr int VPL = kPage / TPV;  // value tokens per lane per page
+  static constexpr int SH = NG == 32 ? 7 : NG == 16 ? 6 : 5;   // log2 of a histogram row in bytes
+  static constexpr int PAGE = NG * kPage;  // bytes of one K (or V) page
   static constexpr int STAGE = (kChunk / kPage) * PAGE;
   static constexpr int KS = kEntries * D * 2;                     // one step slice, K or V
+  static constexpr int HB = kEntries * NG * 4;                    // histogram [256][n_g] u32
+  static constexpr int NPAIR = D / 2;                             // channel pairs of the contraction
+  static constexpr int NREP = kCT / NPAIR;                        // entry phases of the contraction
   static constexpr int OFF_V = KS;
-  static constexpr int OFF_RING = 2 * KS;
-  static constexpr int OFF_PW = OFF_RING + kStages * STAGE;       // per-warp (p, p) pairs of a page
-  static constexpr int OFF_ZQ = OFF_PW + kCW * kPage * 8;
-  static constexpr int OFF_RED = OFF_ZQ + F * 8;
+  static constexpr int OFF_H = 2 * KS;
+  static constexpr int OFF_RING = OFF_H + HB;
+  static constexpr int OFF_ZQ = OFF_RING + kStages * STAGE;
+  static constexpr int OFF_TAB = OFF_ZQ + F * 8;                  // e^{-i TQ theta_f}, e^{-i 480 theta_f}
+  static constexpr int OFF_RED = OFF_TAB + 2 * F * 8;
   static constexpr int OFF_MISC = OFF_RED + 64 * 4;
-  static constexpr int OFF_BAR = OFF_MISC + 16;
-  static constexpr int SMEM = OFF_BAR + 8 * (2 * kStages + 1) + 8;
+  static constexpr int OFF_BAR = OFF_MISC + 32;
+  static constexpr int NBAR = 3 + 2 * kStages;
+  static constexpr int OFF_SC = OFF_BAR + (NBAR * 8 + 15) / 16 * 16;
+  static constexpr int NSC_FIT = (kSmemMax - OFF_SC) / 4 / kChunk;
+  static constexpr int NSC = (NSC_FIT < kMaxSuperChunks ? NSC_FIT : kMaxSuperChunks) * kChunk;
+  static constexpr int SMEM = OFF_SC + NSC * 4;
   static_assert(NP >= 4 && NP <= 32 && 32 % NP == 0, "pair-group mapping");
-  static_assert(NG <= 32 && 32 % NG == 0, "value mapping");
-  static_assert(SMEM <= 227 * 1024, "shared memory");
-  static_assert(OFF_RING % 16 == 0 && OFF_PW % 16 == 0, "alignment");
-  static_assert(kStages * STAGE >= kCW * (D + 2) * 4, "warp partials fit in the ring");
+  static_assert(NG >= 8 && NG <= 32 && 32 % NG == 0, "value mapping");
+  static_assert((1 << SH) == NG * 4, "histogram row");
+  static_assert(NSC >= kChunk && SMEM <= kSmemMax, "shared memory");
+  static_assert(NSC >= 3 * 512 && NSC * 4 >= NREP * NPAIR * 8, "scratch in the score array");
+  static_assert(HB >= kThr * 4, "bf16 reduction in the histogram");
+  static_assert(OFF_RING % 16 == 0 && OFF_SC % 16 == 0 && OFF_BAR % 8 == 0, "alignment");
 };
 
 __device__ inline float2 cmul(float2 a, float2 b) {
@@ -148,7 +171,8 @@ struct Lane {
   int P, tq;
   uint32_t gb_lo, gb_hi;              // byte offsets of the lane's two groups inside a slice row
   uint32_t sel[2];
-  float2 twoc[C], etq[C];
+  int i_own;                          // index, among the lane's tokens of a page, of the one it ends up holding
+  float2 twoc[C], mtwoc[C];           // (2 cos, 2 cos) and its negation, of the lane's token stride
 };
 
 template <int D, int C>
@@ -166,15 +190,23 @@ __device__ inline void lane_init(Lane<D, C>& L, int lane, const float* rope, int
     const int f = L.P * C + e;
     const float2 r = rope_at(rope, RC, F, TQ, f);
     L.twoc[e] = make_float2(2.f * r.x, 2.f * r.x);
-    L.etq[e] = cconj(r);
+    L.mtwoc[e] = make_float2(-2.f * r.x, -2.f * r.x);
   }
+  L.i_own = L.P / X::GRP;
 }
 
 // Scores of the 8 tokens of one page.  On return the lane holds the score of
-// token t_own = tq + TQ * (P / GRP); W advances by TPL tokens.
+// token t_own = tq + TQ * (P / GRP).  With n counting the lane's tokens from the
+// chunk start, the state (Wc, Wn) holds X_n = s_n W_n and X_{n+1}, where
+// s_n = +1, +1, -1, -1, ... (period 4): then X_{n+2} = k X_{n+1} + X_n with
+// k = +2 cos(s theta) for odd n and -2 cos(s theta) for even n -- no negated
+// operand -- and the token's score is s_n times the dot product with X_n.  `ph` is
+// n mod 4 of the page's first token.  With one token per lane per page (TPL = 1)
+// the state is plain W_n and W_{n+2} = 2 cos W_{n+1} - W_n.  The state moves on by
+// TPL tokens.
 template <int D, int C>
 __device__ inline float page_scores(const Lane<D, C>& L, const unsigned char* Ks, const unsigned char* pg,
-                                    float2 (&Wc)[C], float2 (&Wn)[C]) {
+                                    float2 (&Wc)[C], float2 (&Wn)[C], int ph) {
   using X = Dec<D, C>;
   constexpr int TQ = X::TQ, TPL = X::TPL, NP = X::NP;
   const uint2 wlo = *reinterpret_cast<const uint2*>(pg + L.P * kPage);
@@ -205,7 +237,11 @@ __device__ inline float page_scores(const Lane<D, C>& L, const unsigned char* Ks
     acc[i] = a2.x + a2.y;
 #pragma unroll
     for (int e = 0; e < C; ++e) {
-      const float2 nx = __ffma2_rn(L.twoc[e], Wn[e], make_float2(-Wc[e].x, -Wc[e].y));
+      float2 nx;
+      if constexpr (TPL >= 2)       // the page starts at even n: n + i is odd exactly for odd i
+        nx = __ffma2_rn((i & 1) ? L.twoc[e] : L.mtwoc[e], Wn[e], Wc[e]);
+      else
+        nx = __ffma2_rn(L.twoc[e], Wn[e], make_float2(-Wc[e].x, -Wc[e].y));
       Wc[e] = Wn[e];
       Wn[e] = nx;
     }
@@ -230,33 +266,192 @@ __device__ inline float page_scores(const Lane<D, C>& L, const unsigned char* Ks
       acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], o);
     }
   }
+  if constexpr (TPL >= 2) return ((ph + L.i_own) & 2) ? -acc[0] : acc[0];
   return acc[0];
 }
 
-// o += p_t * V_slice[code_t][g] over the lane's tokens of one page.
+// Barrier of the compute warps only (the producer warp never joins it).
+__device__ inline void compute_sync() {
+  asm volatile("bar.sync %0, %1;" :: "r"(kBarCompute), "r"(kCT) : "memory");
+}
+// The same barrier, returning the OR of `v` over the compute threads.
+__device__ inline bool compute_sync_or(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 q, %1, 0;\n bar.red.or.pred p, %2, %3, q;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(r) : "r"((uint32_t)v), "r"(kBarCompute), "r"(kCT) : "memory");
+  return r != 0;
+}
+
+__device__ inline uint32_t warp_sum_u32(uint32_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ inline void red_add_shared(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared.add.u32 [%0], %1;" :: "r"(addr), "r"(v) : "memory");
+}
+
+// Adds the weights of the lane's value tokens of one page to the histogram:
+// H[code][g] += w.  `pg` points at the lane's first code byte, `pw` at its
+// first weight; `hl` is the shared address of H[0][g].
 template <int D, int C>
-__device__ inline void page_values(const unsigned char* Vsm, const unsigned char* pg, const float2* pw2, int gv,
-                                   int tp, uint32_t gbv, float2 (&o)[C / 2]) {
+__device__ inline void hist_page(const unsigned char* pg, const uint32_t* pw, uint32_t hl) {
   using X = Dec<D, C>;
-  constexpr int NG = X::NG, TPV = X::TPV, VPL = X::VPL;
-  const uint2 wv = *reinterpret_cast<const uint2*>(pg + NG * kPage + gv * kPage);
-#pragma unroll
-  for (int jv = 0; jv < VPL; ++jv) {
-    const int t = tp + TPV * jv;
-    uint32_t word, sel;
-    if constexpr (TPV == 1) {
-      word = jv < 4 ? wv.x : wv.y;
-      sel = row_sel(jv);
-    } else {
-      word = t < 4 ? wv.x : wv.y;
-      sel = row_sel(t);
-    }
-    uint32_t v[C / 2];
-    load_row<C>(Vsm, row_addr<D>(word, gbv, sel), v);
-    const float2 p2 = pw2[t];
-#pragma unroll
-    for (int w = 0; w < C / 2; ++w) o[w] = __ffma2_rn(p2, make_float2(bf16_lo(v[w]), bf16_hi(v[w])), o[w]);
+  constexpr int VPL = X::VPL, SH = X::SH;
+  uint32_t cw[2], w[8];
+  if constexpr (VPL == 8) {
+    const uint2 c = *reinterpret_cast<const uint2*>(pg);
+    cw[0] = c.x; cw[1] = c.y;
+    const uint4 a = *reinterpret_cast<const uint4*>(pw);
+    const uint4 b = *reinterpret_cast<const uint4*>(pw + 4);
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w; w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  } else if constexpr (VPL == 4) {
+    cw[0] = *reinterpret_cast<const uint32_t*>(pg);
+    const uint4 a = *reinterpret_cast<const uint4*>(pw);
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+  } else {
+    cw[0] = *reinterpret_cast<const uint16_t*>(pg);
+    const uint2 a = *reinterpret_cast<const uint2*>(pw);
+    w[0] = a.x; w[1] = a.y;
   }
+#pragma unroll
+  for (int k = 0; k < VPL; ++k) {
+    const uint32_t code = __byte_perm(cw[k >> 2], 0u, 0x4440u | (uint32_t)(k & 3));
+    red_add_shared(hl + (code << SH), w[k]);
+  }
+}
+
+constexpr int kBf16Batch = 60;               // bf16 tokens staged at once in the value-slice area
+
+// Non-blocking test of an mbarrier phase.
+__device__ inline bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+__device__ inline void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// This CTA's share of the bf16 tokens (list entries j, j + ns, ... of [sink tokens,
+// recent tokens]), computed by one warp.  Per batch of up to 60 tokens the key and
+// value rows and the coarse RoPE rows of their positions, plus (once) the fine RoPE
+// rows, are bulk-copied into `area` (the value-slice area, free until then); the
+// warp scores each token against the query rotated to its position, keeps an online
+// softmax across batches and writes the partial (o, m, l) to `part`.  Returns true if
+// a wait timed out (the outcome is uniform over the warp).  misc[4] counts the
+// batches whose copies were issued.  `service()` is called between the steps (and
+// while the copies are awaited) so that the warp keeps feeding the code-page ring.
+template <int D, int C, class Service>
+__device__ bool bf16_share(Service& service, const Geo& g, int layer, int step, int b, int h, int j, int ns, int S_eff, int Lc,
+                           int nbj, const __nv_bfloat16* __restrict__ sink, const __nv_bfloat16* __restrict__ ring,
+                           const float* __restrict__ rope, const float2* zq, unsigned char* area, uint32_t bar,
+                           float* part, int* misc) {
+  constexpr int F = D / 2, FPL = F / 32, CPL = D / 32, BB = kBf16Batch;
+  static_assert(8 * F * 8 + BB * (F * 8 + 4 * D) <= kEntries * D * 2, "bf16 batch fits the value-slice area");
+  const int lane = threadIdx.x & 31;
+  float2* fine_s = reinterpret_cast<float2*>(area);                        // [8][F]
+  float2* coarse_s = fine_s + 8 * F;                                       // [BB][F]
+  __nv_bfloat16* kb = reinterpret_cast<__nv_bfloat16*>(coarse_s + BB * F);  // [BB][D]
+  __nv_bfloat16* vb = kb + BB * D;                                         // [BB][D]
+  auto pos_of = [&](int k) { const int i = j + k * ns; return i < S_eff ? i : g.S + Lc + (i - S_eff); };
+  auto row_of = [&](int k, int kv) -> const __nv_bfloat16* {
+    const int i = j + k * ns;
+    if (i < S_eff) return sink + sink_off(g, layer, kv, step, b, h, i);
+    return ring + ring_off(g, layer, kv, step, b, h, (pos_of(k) - g.S) % g.R);
+  };
+  bool to = false;
+  float m = -INFINITY, l = 0.f, o[CPL];
+#pragma unroll
+  for (int u = 0; u < CPL; ++u) o[u] = 0.f;
+  int batch = 0;
+  for (int k0 = 0; k0 < nbj && !to; k0 += BB, ++batch) {
+    const int nbb = min(BB, nbj - k0);
+    if (batch > 0) fence_proxy_async();          // this warp's reads of the area precede the new copies
+    if (lane == 0) {
+      mbar_expect_tx(bar, (batch == 0 ? 8 * F * 8 : 0) + nbb * (F * 8 + 4 * D));
+      misc[4] = batch + 1;
+    }
+    __syncwarp();
+    if (batch == 0 && lane == 0)
+      bulk_g2s(smem_addr(fine_s), rope + (size_t)g.RC * F * 2, 8 * F * 8, bar);
+    for (int k = lane; k < nbb; k += 32) {
+      bulk_g2s(smem_addr(coarse_s + k * F), rope + (size_t)(pos_of(k0 + k) >> 3) * F * 2, F * 8, bar);
+      bulk_g2s(smem_addr(kb + k * D), row_of(k0 + k, 0), D * 2, bar);
+      bulk_g2s(smem_addr(vb + k * D), row_of(k0 + k, 1), D * 2, bar);
+    }
+    {
+      bool done = false;
+      for (long it = 0; it < kWaitIters && !done; ++it) {
+        done = __all_sync(0xffffffffu, mbar_test(bar, batch & 1));
+        if (!done) service();
+      }
+      to = !done;
+    }
+    if (to) break;
+    service();
+    // scores: four tokens at a time, lanes over frequencies; lane (k % 32) keeps token k's
+    float sc0 = -INFINITY, sc1 = -INFINITY;
+    for (int k4 = 0; k4 < nbb; k4 += 4) {
+      float acc[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int k = min(k4 + t, nbb - 1);
+        const int p7 = pos_of(k0 + k) & 7;
+        acc[t] = 0.f;
+#pragma unroll
+        for (int u = 0; u < FPL; ++u) {
+          const int f = lane + 32 * u;
+          const float2 w = cmul(zq[f], cconj(cmul(coarse_s[k * F + f], fine_s[p7 * F + f])));
+          acc[t] = fmaf(w.x, __bfloat162float(kb[k * D + f]), acc[t]);
+          acc[t] = fmaf(w.y, __bfloat162float(kb[k * D + f + F]), acc[t]);
+        }
+      }
+#pragma unroll
+      for (int o2 = 16; o2 > 0; o2 >>= 1)
+#pragma unroll
+        for (int t = 0; t < 4; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o2);
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int k = k4 + t;
+        if (k < nbb && (k & 31) == lane) {
+          if (k < 32) sc0 = acc[t];
+          else sc1 = acc[t];
+        }
+      }
+      service();
+    }
+    // online softmax across batches
+    const float m_new = fmaxf(m, warp_max(fmaxf(sc0, sc1)));
+    const float a_old = l > 0.f ? exp2f(m - m_new) : 0.f;
+    const float p0 = lane < nbb ? exp2f(sc0 - m_new) : 0.f;
+    const float p1 = lane + 32 < nbb ? exp2f(sc1 - m_new) : 0.f;
+    l = l * a_old + warp_sum(p0 + p1);
+#pragma unroll
+    for (int u = 0; u < CPL; ++u) o[u] *= a_old;
+    for (int k = 0; k < nbb; ++k) {
+      const float pk = __shfl_sync(0xffffffffu, k < 32 ? p0 : p1, k & 31);
+#pragma unroll
+      for (int u = 0; u < CPL; ++u) o[u] = fmaf(pk, __bfloat162float(vb[k * D + lane + 32 * u]), o[u]);
+    }
+    m = m_new;
+    service();
+  }
+  fence_proxy_async();                           // the value slice is copied into the area next
+  __syncwarp();
+#pragma unroll
+  for (int u = 0; u < CPL; ++u) part[lane + 32 * u] = to ? 0.f : o[u];
+  if (lane == 0) {
+    part[D] = to || l == 0.f ? -INFINITY : m;
+    part[D + 1] = to ? 0.f : l;
+  }
+  return to;
 }
 
 template <int D, int C>
@@ -268,25 +463,32 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
     float* __restrict__ ws, float* __restrict__ out, float* __restrict__ lse, float* __restrict__ split_lse,
     int32_t* st) {
   using X = Dec<D, C>;
-  constexpr int F = X::F, NG = X::NG, TQ = X::TQ, GRP = X::GRP, TPV = X::TPV;
+  constexpr int F = X::F, NG = X::NG, TQ = X::TQ, GRP = X::GRP, NPAIR = X::NPAIR, NREP = X::NREP;
   extern __shared__ __align__(1024) unsigned char smem[];
   unsigned char* Ks = smem;
-  unsigned char* Vsm = smem + X::OFF_V;
+  const unsigned char* Vsm = smem + X::OFF_V;
+  uint32_t* Hs = reinterpret_cast<uint32_t*>(smem + X::OFF_H);
   unsigned char* ringb = smem + X::OFF_RING;
-  float2* pwall = reinterpret_cast<float2*>(smem + X::OFF_PW);
   float2* zq = reinterpret_cast<float2*>(smem + X::OFF_ZQ);
+  float2* etq_s = reinterpret_cast<float2*>(smem + X::OFF_TAB);       // [F] e^{-i TQ theta_f}
+  float2* ech_s = etq_s + F;                                           // [F] e^{-i kChunk theta_f}
   float* red = reinterpret_cast<float*>(smem + X::OFF_RED);
-  int* misc = reinterpret_cast<int*>(smem + X::OFF_MISC);        // [0]: failure flag, [1]: merge flag
+  // misc: [0] failure, [1] merger, [2] chunks issued, [3] V slice issued, [4] bf16 batches issued
+  int* misc = reinterpret_cast<int*>(smem + X::OFF_MISC);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + X::OFF_BAR);
-  // bars[0]: slices (or the bf16 tokens); bars[1 + s]: stage s full; bars[1 + kStages + s]: stage s empty
+  float* SC = reinterpret_cast<float*>(smem + X::OFF_SC);    // scores, then weights; scratch elsewhere
+  // bars[0]: K slice; bars[1]: V slice; bars[2 + s]: stage s full; bars[2 + kStages + s]: stage s empty;
+  // bars[2 + 2 kStages]: the bf16 rows
 
   const int j = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
   const int h = hq / (g.Hq / g.H);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool producer = warp == kCW;
   const int blk = step / g.Tc, s = step % g.Tc;
-  const size_t slot_base = ((size_t)b * g.Hq + hq) * (g.max_splits + 1);
-  int32_t* counters = reinterpret_cast<int32_t*>(ws + (size_t)g.B * g.Hq * (g.max_splits + 1) * (D + 2));
+  const size_t slot0 = ((size_t)b * g.Hq + hq) * g.max_splits * 2;        // partial slots [split][coded, bf16]
+  float* part_coded = ws + (slot0 + 2 * j) * (D + 2);
+  float* part_bf16 = ws + (slot0 + 2 * j + 1) * (D + 2);
+  int32_t* counters = reinterpret_cast<int32_t*>(ws + (size_t)g.B * g.Hq * g.max_splits * 2 * (D + 2));
 
   const int ctx = ctx_len[b], Lc = coded_len[b];
   const int S_eff = min(g.S, max(ctx, 0));
@@ -297,335 +499,350 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
 
   int chunk = (Lc + ns - 1) / ns;
   chunk = (chunk + 31) & ~31;
-  const int n0 = (bad || j >= ns) ? 0 : min(Lc, j * chunk);
-  const int n1 = (bad || j >= ns) ? 0 : min(Lc, n0 + chunk);
+  const int n0 = bad ? 0 : min(Lc, j * chunk);
+  const int n1 = bad ? 0 : min(Lc, n0 + chunk);
   const bool do_coded = n0 < n1;
-  const int n_chunks = do_coded ? (n1 - n0 + kChunk - 1) / kChunk : 0;
-  const uint8_t* pages = idx + idx_page_off(g, layer, blk, b, h, 0);
+  const int n_kchunks = do_coded ? (n1 - n0 + kChunk - 1) / kChunk : 0;
+  const int n_stream = 2 * n_kchunks;            // per super-chunk: its K chunks, then its V chunks
+  const int n_super = do_coded ? (n1 - n0 + X::NSC - 1) / X::NSC : 0;
+  constexpr int CPS = X::NSC / kChunk;           // chunks per full super-chunk
+  const uint8_t* kstream = idx + idx_stream_off(g, layer, blk, b, h, 0);
+  const uint8_t* vstream = idx + idx_stream_off(g, layer, blk, b, h, 1);
+
+  // the V slice is needed only by the first contraction: the producer copies it once its bf16 share
+  // (staged in the same area) is done
+  auto issue_v_slice = [&]() {
+    const uint32_t bv = smem_addr(&bars[1]);
+    mbar_expect_tx(bv, X::KS);
+    bulk_g2s(smem_addr(Vsm), cbp + cbp_slice_off(g, layer, 1, blk, h, s), X::KS, bv);
+  };
+  // chunk `ci` of the stream: its first coded token and which half of the page stream it reads
+  auto issue_chunk = [&](int ci) {
+    const int sc = ci / (2 * CPS), r = ci % (2 * CPS);
+    const int nk = min(CPS, n_kchunks - sc * CPS);
+    const bool is_v = r >= nk;
+    const int c0 = n0 + (sc * CPS + (is_v ? r - nk : r)) * kChunk;
+    const int np = (min(n1, c0 + kChunk) - c0 + kPage - 1) / kPage;
+    const uint32_t bar = smem_addr(&bars[2 + ci % kStages]);
+    mbar_expect_tx(bar, np * X::PAGE);
+    bulk_g2s(smem_addr(ringb + (ci % kStages) * X::STAGE), (is_v ? vstream : kstream) + (size_t)(c0 / kPage) * X::PAGE,
+             np * X::PAGE, bar);
+  };
 
   if (tid == 0) {
-    mbar_init(smem_addr(&bars[0]), 1);
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(smem_addr(&bars[1 + i]), 1);
-      mbar_init(smem_addr(&bars[1 + kStages + i]), kCW);
-    }
+    for (int i = 0; i < X::NBAR; ++i) mbar_init(smem_addr(&bars[i]), i >= 2 + kStages && i < 2 + 2 * kStages ? kCW : 1);
     fence_mbar_init();
     misc[0] = 0;
     misc[1] = 0;
+    misc[2] = 0;
+    misc[3] = 0;
+    misc[4] = 0;
   }
-  // query rotated at its own position, scaled so scores come out in log2 units
-  if (!bad) {
-    const int qpos = ctx - 1;
-    const float qscale = 1.4426950408889634f * rsqrtf((float)D);
+  __syncthreads();
+  // ---- prologue: the producer starts the K slice and the first chunks; compute threads rotate the
+  // query (scaled so that scores come out in log2 units) and clear the histogram
+  const int nb = bad ? 0 : S_eff + recent;                 // bf16 tokens: [sink tokens, recent tokens]
+  const int nbj = nb > j ? (nb - j + ns - 1) / ns : 0;    // this CTA's share: j, j + ns, ...
+  if (producer && lane == 0 && do_coded) {
+    const uint32_t bk = smem_addr(&bars[0]);
+    mbar_expect_tx(bk, X::KS);
+    bulk_g2s(smem_addr(Ks), cbp + cbp_slice_off(g, layer, 0, blk, h, s), X::KS, bk);
+    for (int ci = 0; ci < min(kStages, n_stream); ++ci) issue_chunk(ci);
+  }
+  if (!bad && tid < F) {
     const __nv_bfloat16* qv = q + ((size_t)b * g.Hq + hq) * D;
-    for (int f = tid; f < F; f += blockDim.x) {
-      const float2 e = rope_at(rope, g.RC, F, qpos, f);
-      const float a = __bfloat162float(qv[f]), c2 = __bfloat162float(qv[f + F]);
-      zq[f] = make_float2((a * e.x - c2 * e.y) * qscale, (c2 * e.x + a * e.y) * qscale);
-    }
+    const float2 qraw = make_float2(__bfloat162float(qv[tid]), __bfloat162float(qv[tid + F]));
+    const float2 qe = rope_at(rope, g.RC, F, ctx - 1, tid);
+    const float2 e_tq = rope_at(rope, g.RC, F, X::TQ, tid);
+    const float2 e_ch = rope_at(rope, g.RC, F, kChunk, tid);
+    const float qscale = 1.4426950408889634f * rsqrtf((float)D);
+    zq[tid] = make_float2((qraw.x * qe.x - qraw.y * qe.y) * qscale, (qraw.y * qe.x + qraw.x * qe.y) * qscale);
+    etq_s[tid] = cconj(e_tq);
+    ech_s[tid] = cconj(e_ch);
   }
+  if (!producer)
+    for (int i = tid; i < X::HB / 16; i += kCT) reinterpret_cast<uint4*>(Hs)[i] = make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
 
   bool timed_out = false;
-  float m_w = -INFINITY, l_w = 0.f;       // warp's reference maximum (log2) and weight sum (writer lanes)
-  float2 o[C / 2];
-#pragma unroll
-  for (int w = 0; w < C / 2; ++w) o[w] = make_float2(0.f, 0.f);
+  float m_run = -INFINITY, l_run = 0.f;       // the coded partial, held by compute threads tid < NPAIR
+  float2 o_run = make_float2(0.f, 0.f);
 
   if (do_coded) {
     if (producer) {
-      // ---- producer: the two step slices, then the chunks through the ring
+      // ---- producer: the bf16 share, feeding the ring meanwhile (lane 0 issues every chunk whose
+      // stage its consumers have released); the V slice into the area the share used; then the
+      // rest of the chunks
+      int ci_next = min(kStages, n_stream);
+      auto service = [&]() {
+        if (lane == 0)
+          while (ci_next < n_stream &&
+                 mbar_test(smem_addr(&bars[2 + kStages + ci_next % kStages]), (ci_next / kStages - 1) & 1))
+            issue_chunk(ci_next++);
+      };
+      timed_out = bf16_share<D, C>(service, g, layer, step, b, h, j, ns, S_eff, Lc, nbj, sink, ring, rope, zq,
+                                   smem + X::OFF_V, smem_addr(&bars[2 + 2 * kStages]), part_bf16, misc);
+      if (lane == 0 && !timed_out) {
+        issue_v_slice();
+        misc[3] = 1;
+      }
       if (lane == 0) {
-        const uint32_t bar0 = smem_addr(&bars[0]);
-        mbar_expect_tx(bar0, 2 * X::KS);
-        bulk_g2s(smem_addr(Ks), cbp + cbp_slice_off(g, layer, 0, blk, h, s), X::KS, bar0);
-        bulk_g2s(smem_addr(Vsm), cbp + cbp_slice_off(g, layer, 1, blk, h, s), X::KS, bar0);
-        for (int ci = 0; ci < n_chunks; ++ci) {
-          if (ci >= kStages &&
-              !mbar_wait(smem_addr(&bars[1 + kStages + ci % kStages]), (ci / kStages - 1) & 1, kWaitIters)) {
+        int ci = ci_next;
+        for (; ci < n_stream; ++ci) {
+          if (!mbar_wait(smem_addr(&bars[2 + kStages + ci % kStages]), (ci / kStages - 1) & 1, kWaitIters)) {
             timed_out = true;
             break;
           }
-          const int c0 = n0 + ci * kChunk;
-          const int np = (min(n1, c0 + kChunk) - c0 + kPage - 1) / kPage;
-          const uint32_t bar = smem_addr(&bars[1 + ci % kStages]);
-          mbar_expect_tx(bar, np * X::PAGE);
-          bulk_g2s(smem_addr(ringb + (ci % kStages) * X::STAGE), pages + (size_t)(c0 / kPage) * X::PAGE,
-                   np * X::PAGE, bar);
+          issue_chunk(ci);
         }
+        misc[2] = ci;
       }
     } else {
       // ---- compute warps
       Lane<D, C> L;
       lane_init<D, C>(L, lane, rope, g.RC);
-      float2 echunk[C], U[C];
+      float2 U[C];                       // W of the lane's first token of the current chunk
       const int p_first = g.S + n0 + kPage * kPPW * warp + L.tq;
 #pragma unroll
       for (int e = 0; e < C; ++e) {
         const int f = L.P * C + e;
-        echunk[e] = cconj(rope_at(rope, g.RC, F, kChunk, f));
         U[e] = cmul(zq[f], cconj(rope_at(rope, g.RC, F, p_first, f)));
       }
-      float2* pw2 = pwall + warp * kPage;
       const bool writer = (L.P % GRP) == 0;
       const int t_own = L.tq + TQ * (L.P / GRP);
       const int gv = lane % NG, tp = lane / NG;
-      const uint32_t gbv = (uint32_t)gv * C * 2;
-      // waits are bounded; their outcome is made uniform over the warp
+      const uint32_t hl = smem_addr(Hs) + (uint32_t)gv * 4;
+      uint32_t* PW = reinterpret_cast<uint32_t*>(SC);
+      // waits are bounded; their outcome is made uniform over the warp, then over the compute warps
       timed_out = __any_sync(0xffffffffu, !mbar_wait(smem_addr(&bars[0]), 0, kWaitIters));
-
-      for (int ci = 0; ci < n_chunks && !timed_out; ++ci) {
-        const int c0 = n0 + ci * kChunk;
-        timed_out = __any_sync(0xffffffffu, !mbar_wait(smem_addr(&bars[1 + ci % kStages]), (ci / kStages) & 1,
-                                                       kWaitIters));
-        if (timed_out) break;
-        const unsigned char* stage = ringb + (ci % kStages) * X::STAGE;
-        float2 Wc[C], Wn[C];
+      int ci = 0;
+      for (int sc = 0; sc < n_super; ++sc) {
+        const int s0 = n0 + sc * X::NSC, s1 = min(n1, s0 + X::NSC);
+        const int nk = (s1 - s0 + kChunk - 1) / kChunk;
+        // ---- phase A: scores of the super-chunk
+        float mx = -INFINITY;
+        for (int kc = 0; kc < nk; ++kc, ++ci) {
+          if (!timed_out)
+            timed_out = __any_sync(0xffffffffu, !mbar_wait(smem_addr(&bars[2 + ci % kStages]), (ci / kStages) & 1,
+                                                           kWaitIters));
+          if (!timed_out) {
+            const int c0 = s0 + kc * kChunk;
+            const unsigned char* stage = ringb + (ci % kStages) * X::STAGE;
+            float2 Wc[C], Wn[C];
 #pragma unroll
-        for (int e = 0; e < C; ++e) { Wc[e] = U[e]; Wn[e] = cmul(U[e], L.etq[e]); }
-#pragma unroll 1
-        for (int pi = 0; pi < kPPW; ++pi) {
-          const int pl = warp * kPPW + pi;
-          const int tb = c0 + kPage * pl;
-          if (tb >= n1) break;
-          const unsigned char* pg = stage + pl * X::PAGE;
-          const float sc = page_scores<D, C>(L, Ks, pg, Wc, Wn);
-          const bool valid = tb + t_own < n1;
-          const float sv = valid ? sc : -INFINITY;
-          // online softmax per warp: raise the reference only when a score passes it by 2^16
-          if (__any_sync(0xffffffffu, sv > m_w + kRaiseLog2)) {
-            const float m_new = fmaxf(m_w, warp_max(sv));
-            const float alpha = exp2f(m_w - m_new);     // 0 for the first page
+            for (int e = 0; e < C; ++e) {
+              Wc[e] = U[e];
+              Wn[e] = cmul(U[e], etq_s[L.P * C + e]);     // s_1 = +1
+            }
+#pragma unroll 2
+            for (int pi = 0; pi < kPPW; ++pi) {
+              const int pl = warp * kPPW + pi;
+              const int tb = c0 + kPage * pl;
+              if (tb >= s1) break;
+              const float sc_ = page_scores<D, C>(L, Ks, stage + pl * X::PAGE, Wc, Wn, (pi * X::TPL) & 3);
+              const float sv = tb + t_own < s1 ? sc_ : -INFINITY;
+              mx = fmaxf(mx, sv);
+              if (writer) SC[tb - s0 + t_own] = sv;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&bars[2 + kStages + ci % kStages]));
+          }
 #pragma unroll
-            for (int w = 0; w < C / 2; ++w) o[w] = make_float2(o[w].x * alpha, o[w].y * alpha);
-            l_w *= alpha;
-            m_w = m_new;
-          }
-          const float p = valid ? exp2f(sv - m_w) : 0.f;
-          if (writer) {
-            pw2[t_own] = make_float2(p, p);
-            l_w += p;
-          }
-          __syncwarp();
-          page_values<D, C>(Vsm, pg, pw2, gv, tp, gbv, o);
-          __syncwarp();
+          for (int e = 0; e < C; ++e) U[e] = cmul(U[e], ech_s[L.P * C + e]);
         }
-        if (lane == 0) mbar_arrive(smem_addr(&bars[1 + kStages + ci % kStages]));
+        // ---- weights: exact maximum, then integers round(2^(s - M) * 2^k) with 2^k * sum < 2^30
+        mx = warp_max(mx);
+        if (lane == 0) red[warp] = mx;
+        timed_out = compute_sync_or(timed_out);
+        float M = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < C; ++e) U[e] = cmul(U[e], echunk[e]);
+        for (int w = 0; w < kCW; ++w) M = fmaxf(M, red[w]);
+        const int len = s1 - s0, len8 = (len + kPage - 1) & ~(kPage - 1);
+        float ls = 0.f;
+        if (!timed_out)
+#pragma unroll 4
+          for (int t = tid; t < len; t += kCT) {
+            const float p = exp2f(SC[t] - M);
+            SC[t] = p;
+            ls += p;
+          }
+        ls = warp_sum(ls);
+        if (lane == 0) red[16 + warp] = ls;
+        compute_sync();
+        float Ls = 0.f;
+#pragma unroll
+        for (int w = 0; w < kCW; ++w) Ls += red[16 + w];
+        // Ls = m 2^E with m in [0.5, 1); Ls >= 1 (the maximum's weight is 1), so 17 <= 30 - E <= 29
+        const int E = ((__float_as_int(Ls) >> 23) & 0xff) - 126;
+        const int kfx = min(30, max(0, 30 - E));
+        const float scale = __int_as_float((127 + kfx) << 23);
+        uint32_t lf = 0;
+        if (!timed_out)
+#pragma unroll 4
+          for (int t = tid; t < len8; t += kCT) {
+            const uint32_t v = t < len ? __float2uint_rn(SC[t] * scale) : 0u;
+            PW[t] = v;
+            lf += v;
+          }
+        lf = warp_sum_u32(lf);
+        if (lane == 0) reinterpret_cast<uint32_t*>(red)[32 + warp] = lf;
+        compute_sync();
+        uint32_t Lf = 0;
+#pragma unroll
+        for (int w = 0; w < kCW; ++w) Lf += reinterpret_cast<uint32_t*>(red)[32 + w];
+        // ---- phase B: histogram of the weights over (code, group)
+        for (int kc = 0; kc < nk; ++kc, ++ci) {
+          if (!timed_out)
+            timed_out = __any_sync(0xffffffffu, !mbar_wait(smem_addr(&bars[2 + ci % kStages]), (ci / kStages) & 1,
+                                                           kWaitIters));
+          if (timed_out) continue;
+          const int c0 = s0 + kc * kChunk;
+          const unsigned char* stage = ringb + (ci % kStages) * X::STAGE;
+#pragma unroll 2
+          for (int pi = 0; pi < kPPW; ++pi) {
+            const int pl = warp * kPPW + pi;
+            const int tb = c0 + kPage * pl;
+            if (tb >= s1) break;
+            hist_page<D, C>(stage + pl * X::PAGE + gv * kPage + tp * X::VPL, PW + (tb - s0) + tp * X::VPL, hl);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_addr(&bars[2 + kStages + ci % kStages]));
+        }
+        if (!timed_out && sc == 0)
+          timed_out = __any_sync(0xffffffffu, !mbar_wait(smem_addr(&bars[1]), 0, kWaitIters));
+        timed_out = compute_sync_or(timed_out);
+        // ---- contraction: o[ch] = sum_a H[a][ch / c] * V[a][ch], two channels per thread
+        const int cp = tid % NPAIR, rep = tid / NPAIR;
+        float2 acc = make_float2(0.f, 0.f);
+        if (!timed_out && rep < NREP) {
+          const uint32_t* vcol = reinterpret_cast<const uint32_t*>(Vsm) + cp;
+          const uint32_t* hcol = Hs + (2 * cp) / C;
+#pragma unroll 4
+          for (int a = rep; a < kEntries; a += NREP) {
+            const uint32_t v = vcol[a * NPAIR];
+            const float hv = (float)hcol[a * NG];
+            acc.x = fmaf(hv, bf16_lo(v), acc.x);
+            acc.y = fmaf(hv, bf16_hi(v), acc.y);
+          }
+        }
+        float2* rb = reinterpret_cast<float2*>(SC);      // [NREP][NPAIR]: the weights are no longer read
+        if (rep < NREP) rb[rep * NPAIR + cp] = acc;
+        compute_sync();
+        if (tid < NPAIR && !timed_out && Lf > 0u) {
+          float2 o = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int r = 0; r < NREP; ++r) { o.x += rb[r * NPAIR + tid].x; o.y += rb[r * NPAIR + tid].y; }
+          const float sc_scale = __int_as_float((127 - kfx) << 23);
+          const float l_sc = (float)Lf * sc_scale;
+          const float m_new = fmaxf(m_run, M);
+          const float a_old = l_run > 0.f ? exp2f(m_run - m_new) : 0.f;
+          const float a_new = exp2f(M - m_new) * sc_scale;
+          o_run = make_float2(o_run.x * a_old + o.x * a_new, o_run.y * a_old + o.y * a_new);
+          l_run = l_run * a_old + l_sc * exp2f(M - m_new);
+          m_run = m_new;
+        }
+        if (sc + 1 < n_super)
+          for (int i = tid; i < X::HB / 16; i += kCT) reinterpret_cast<uint4*>(Hs)[i] = make_uint4(0u, 0u, 0u, 0u);
+        compute_sync();
       }
     }
   }
+  auto no_service = []() {};
+  if (!do_coded && producer)
+    timed_out = bf16_share<D, C>(no_service, g, layer, step, b, h, j, ns, S_eff, Lc, nbj, sink, ring, rope, zq,
+                                 smem + X::OFF_V, smem_addr(&bars[2 + 2 * kStages]), part_bf16, misc);
   if (__syncthreads_or(timed_out)) {
     if (tid == 0) {
       set_status(st, LVQ_ETIMEOUT);
       misc[0] = 1;
       if (do_coded) {   // let every issued copy land before the CTA can exit
+        const int issued = max(misc[2], min(kStages, n_stream));
         mbar_wait(smem_addr(&bars[0]), 0, kWaitIters);
-        for (int ci = 0; ci < min(n_chunks, kStages); ++ci) mbar_wait(smem_addr(&bars[1 + ci]), 0, kWaitIters);
+        if (misc[3]) mbar_wait(smem_addr(&bars[1]), 0, kWaitIters);
+        for (int ci = max(0, issued - kStages); ci < issued; ++ci)
+          mbar_wait(smem_addr(&bars[2 + ci % kStages]), (ci / kStages) & 1, kWaitIters);
       }
+      if (misc[4] > 0) mbar_wait(smem_addr(&bars[2 + 2 * kStages]), (misc[4] - 1) & 1, kWaitIters);
     }
     __syncthreads();
   }
-
-  // ---- coded partial: combine the warps' (m, l, o) -- staged in the free ring
-  if (j < ns) {
-    float* part = ws + (slot_base + j) * (D + 2);
-    float* wo = reinterpret_cast<float*>(ringb);          // [kCW][D + 2]
-    if (!producer) {
-      // sum the value accumulators over the lanes sharing a group
-#pragma unroll
-      for (int off = NG; off < 32; off <<= 1)
-#pragma unroll
-        for (int w = 0; w < C / 2; ++w) {
-          o[w].x += __shfl_xor_sync(0xffffffffu, o[w].x, off);
-          o[w].y += __shfl_xor_sync(0xffffffffu, o[w].y, off);
-        }
-      const float lsum = warp_sum(l_w);
-      float* mine = wo + warp * (D + 2);
-      if (lane < NG) {
-#pragma unroll
-        for (int w = 0; w < C / 2; ++w) {
-          mine[lane * C + 2 * w] = o[w].x;
-          mine[lane * C + 2 * w + 1] = o[w].y;
-        }
-      }
-      if (lane == 0) { mine[D] = m_w; mine[D + 1] = lsum; }
-    }
-    __syncthreads();
-    const bool ok = do_coded && !misc[0];
-    float M = -INFINITY;
-    for (int w = 0; w < kCW; ++w) M = fmaxf(M, wo[w * (D + 2) + D]);
-    if (tid < D) {
-      float oe = 0.f;
-      if (ok && M != -INFINITY)
-        for (int w = 0; w < kCW; ++w) {
-          const float mw = wo[w * (D + 2) + D];
-          if (mw != -INFINITY) oe = fmaf(exp2f(mw - M), wo[w * (D + 2) + tid], oe);
-        }
-      part[tid] = oe;
-    }
-    if (tid == 0) {
-      float Ls = 0.f;
-      if (ok && M != -INFINITY)
-        for (int w = 0; w < kCW; ++w) {
-          const float mw = wo[w * (D + 2) + D];
-          if (mw != -INFINITY) Ls = fmaf(exp2f(mw - M), wo[w * (D + 2) + D + 1], Ls);
-        }
-      part[D] = ok ? M : -INFINITY;
-      part[D + 1] = ok ? Ls : 0.f;
-    }
+  const bool failed = misc[0] != 0;
+  if (tid < NPAIR) {
+    part_coded[2 * tid] = failed ? 0.f : o_run.x;
+    part_coded[2 * tid + 1] = failed ? 0.f : o_run.y;
+  }
+  if (tid == 0) {
+    part_coded[D] = failed || l_run == 0.f ? -INFINITY : m_run;
+    part_coded[D + 1] = failed ? 0.f : l_run;
   }
 
-  // ---- CTA ns: the bf16 partial (sink tokens and recent window)
-  if (j == ns) {
-    float* pb = ws + (slot_base + ns) * (D + 2);
-    const int nb = bad ? 0 : S_eff + recent;
-    const int nrow = g.S + g.R;
-    __nv_bfloat16* Kb = reinterpret_cast<__nv_bfloat16*>(smem);          // [S + R][D]
-    __nv_bfloat16* Vb = Kb + (size_t)nrow * D;                             // [S + R][D]
-    // RoPE rows: sink positions [0, S) use coarse rows 0..; recent positions use coarse rows r0..r1
-    float2* fine_s = reinterpret_cast<float2*>(Vb + (size_t)nrow * D);    // [8][F]
-    float2* coarse_s = fine_s + 8 * F;                                     // [n_sink_rows + n_rec_rows][F]
-    float* sc = reinterpret_cast<float*>(coarse_s);                        // reused after the scores
-    const int sink_rows = (S_eff + 7) / 8;
-    const int r0 = (g.S + Lc) >> 3, r1 = recent > 0 ? (ctx - 1) >> 3 : r0 - 1;
-    const int rec_rows = r1 - r0 + 1;
-    bool ok = true;
-    if (nb > 0) {
-      const uint32_t barb = smem_addr(&bars[0]);
-      if (tid == 0) {
-        const uint32_t sb = (uint32_t)S_eff * D * 2, rb = (uint32_t)g.R * D * 2;
-        mbar_expect_tx(barb, 2 * (sb + rb));
-        if (sb) {
-          bulk_g2s(smem_addr(Kb), sink + sink_off(g, layer, 0, step, b, h, 0), sb, barb);
-          bulk_g2s(smem_addr(Vb), sink + sink_off(g, layer, 1, step, b, h, 0), sb, barb);
-        }
-        bulk_g2s(smem_addr(Kb + (size_t)g.S * D), ring + ring_off(g, layer, 0, step, b, h, 0), rb, barb);
-        bulk_g2s(smem_addr(Vb + (size_t)g.S * D), ring + ring_off(g, layer, 1, step, b, h, 0), rb, barb);
-      }
-      const float2* rp = reinterpret_cast<const float2*>(rope);
-      for (int i = tid; i < 8 * F; i += blockDim.x) fine_s[i] = rp[(size_t)g.RC * F + i];
-      for (int i = tid; i < sink_rows * F; i += blockDim.x) coarse_s[i] = rp[i];
-      for (int i = tid; i < rec_rows * F; i += blockDim.x) coarse_s[sink_rows * F + i] = rp[(size_t)r0 * F + i];
-      ok = !__syncthreads_or(!mbar_wait(barb, 0, kWaitIters));
-      if (!ok && tid == 0) set_status(st, LVQ_ETIMEOUT);
-    }
-    // scores: 4 threads per token, a quarter of the frequencies each
-    constexpr int FQ = F / 4;
-    float my_sc[4];
-    int n_mine = 0;
-    for (int i0 = 0; i0 < nb && ok; i0 += kThr / 4) {
-      const int i = i0 + tid / 4, qf = tid % 4;
-      float part_s = 0.f;
-      if (i < nb) {
-        int pos, row, crow;
-        if (i < S_eff) { pos = i; row = i; crow = pos >> 3; }
-        else {
-          pos = g.S + Lc + (i - S_eff);
-          row = g.S + (pos - g.S) % g.R;
-          crow = sink_rows + (pos >> 3) - r0;
-        }
-        const __nv_bfloat16* kr = Kb + (size_t)row * D;
-        const float2* cr = coarse_s + (size_t)crow * F;
-        const float2* fr = fine_s + (size_t)(pos & 7) * F;
-#pragma unroll 4
-        for (int f = qf * FQ; f < (qf + 1) * FQ; ++f) {
-          const float2 w = cmul(zq[f], cconj(cmul(cr[f], fr[f])));
-          part_s = fmaf(w.x, __bfloat162float(kr[f]), part_s);
-          part_s = fmaf(w.y, __bfloat162float(kr[f + F]), part_s);
-        }
-      }
-      part_s += __shfl_xor_sync(0xffffffffu, part_s, 1);
-      part_s += __shfl_xor_sync(0xffffffffu, part_s, 2);
-      my_sc[n_mine++ & 3] = part_s;           // the thread's tokens i0/4-stride (at most 4 passes)
-    }
-    // maximum and weights (each token's score lives in its 4 threads)
-    float mloc = -INFINITY;
-    for (int k = 0, i0 = 0; i0 < nb && ok; i0 += kThr / 4, ++k)
-      if (i0 + tid / 4 < nb) mloc = fmaxf(mloc, my_sc[k & 3]);
-    const float M = block_reduce<true>(mloc, red);
-    __syncthreads();                           // the RoPE rows are no longer read: sc may overwrite them
-    float lloc = 0.f;
-    for (int k = 0, i0 = 0; i0 < nb && ok; i0 += kThr / 4, ++k) {
-      const int i = i0 + tid / 4;
-      if (i < nb && (tid % 4) == 0) {
-        const float p = exp2f(my_sc[k & 3] - M);
-        sc[i] = p;
-        lloc += p;
-      }
-    }
-    const float Lb = block_reduce<false>(lloc, red);     // block_reduce syncs: sc holds the weights
-    constexpr int NTS = kThr / D;
-    float ov = 0.f;
-    {
-      const int e = tid % D, ts = tid / D;
-      for (int i = ts; i < nb && ok; i += NTS) {
-        const int row = i < S_eff ? i : g.S + (Lc + (i - S_eff)) % g.R;
-        ov = fmaf(sc[i], __bfloat162float(Vb[(size_t)row * D + e]), ov);
-      }
-    }
-    __syncthreads();
-    float* parts = reinterpret_cast<float*>(smem);      // the staged tokens are no longer read
-    parts[tid] = ov;
-    __syncthreads();
-    if (tid < D) {
-      float oe = 0.f;
-#pragma unroll
-      for (int k2 = 0; k2 < NTS; ++k2) oe += parts[k2 * D + tid];
-      pb[tid] = oe;
-    }
-    if (tid == 0) {
-      const bool any = ok && nb > 0;
-      pb[D] = any ? M : -INFINITY;
-      pb[D + 1] = any ? Lb : 0.f;
-    }
-  }
-
-  // ---- the last CTA of this (request, head) merges the ns + 1 partials
-  __threadfence();
+  // ---- the last CTA of this (request, head) merges the 2 * ns partials
   __syncthreads();
-  if (tid == 0) misc[1] = atomicAdd(&counters[(size_t)b * g.Hq + hq], 1) == ns;
+  if (tid == 0) {
+    __threadfence();            // this CTA's partials (ordered before by the barrier) become visible
+    misc[1] = atomicAdd(&counters[(size_t)b * g.Hq + hq], 1) == ns - 1;
+  }
   __syncthreads();
   if (!misc[1]) return;
   __threadfence();
-  const float* base = ws + slot_base * (D + 2);
-  float* lse2 = red + 32;                     // up to 32 partials via red[], else recomputed below
-  (void)lse2;
-  float M = -INFINITY;
-  for (int i = 0; i <= ns; ++i) {
-    const float* pj = base + (size_t)i * (D + 2);
-    const float l = __ldcg(pj + D + 1);
-    if (l > 0.f) M = fmaxf(M, __ldcg(pj + D) + log2f(l));
+  const int np = 2 * ns;
+  const float* base = ws + slot0 * (D + 2);
+  constexpr int RB = kThr / D;                // partial phases of the output sum
+  constexpr int MPF = 8;                      // output elements prefetched per thread
+  const int e = tid % D, r = tid / D;
+  // every load is issued before the first use: (m, l) of partial tid, and o[e] of partials r, r + RB, ...
+  float pm = -INFINITY, pl = 0.f;
+  if (tid < np) {
+    pm = __ldcg(base + (size_t)tid * (D + 2) + D);
+    pl = __ldcg(base + (size_t)tid * (D + 2) + D + 1);
   }
-  float den = 0.f;
-  if (M != -INFINITY)
-    for (int i = 0; i <= ns; ++i) {
-      const float* pj = base + (size_t)i * (D + 2);
-      const float l = __ldcg(pj + D + 1);
-      if (l > 0.f) den += exp2f(__ldcg(pj + D) + log2f(l) - M);
+  float opre[MPF];
+#pragma unroll
+  for (int u = 0; u < MPF; ++u) {
+    const int i = r + RB * u;
+    opre[u] = i < np ? __ldcg(base + (size_t)i * (D + 2) + e) : 0.f;
+  }
+  float* pl2 = SC;              // [np] partial LSEs (log2)
+  float* pw = SC + 512;         // [np] partial weights
+  const float lse_i = pl > 0.f ? pm + log2f(pl) : -INFINITY;
+  if (tid < np) pl2[tid] = lse_i;
+  const float M = block_reduce<true>(lse_i, red);
+  const float den = block_reduce<false>(M != -INFINITY && lse_i != -INFINITY ? exp2f(lse_i - M) : 0.f, red);
+  const float Ltot = M == -INFINITY ? -INFINITY : M + log2f(den);
+  if (tid < np) pw[tid] = lse_i == -INFINITY ? 0.f : exp2f(pm - Ltot);
+  __syncthreads();
+  {
+    float acc = 0.f;
+#pragma unroll
+    for (int u = 0; u < MPF; ++u) {
+      const int i = r + RB * u;
+      if (i < np) acc = fmaf(pw[i], opre[u], acc);
     }
-  const float L2 = M == -INFINITY ? -INFINITY : M + log2f(den);
-  if (tid < D) {
-    float ov = 0.f;
-    if (M != -INFINITY)
-      for (int i = 0; i <= ns; ++i) {
-        const float* pj = base + (size_t)i * (D + 2);
-        if (__ldcg(pj + D + 1) > 0.f) ov = fmaf(exp2f(__ldcg(pj + D) - L2), __ldcg(pj + tid), ov);
-      }
-    out[((size_t)b * g.Hq + hq) * D + tid] = ov;
+    for (int i = r + RB * MPF; i < np; i += RB) acc = fmaf(pw[i], __ldcg(base + (size_t)i * (D + 2) + e), acc);
+    float* rb = SC + 1024;      // [RB][D]
+    rb[r * D + e] = acc;
+    __syncthreads();
+    if (tid < D) {
+      float t = 0.f;
+#pragma unroll
+      for (int r2 = 0; r2 < RB; ++r2) t += rb[r2 * D + tid];
+      out[((size_t)b * g.Hq + hq) * D + tid] = t;
+    }
   }
   constexpr float kLn2 = 0.6931471805599453f;
   if (tid == 0) {
-    lse[(size_t)b * g.Hq + hq] = L2 * kLn2;
+    lse[(size_t)b * g.Hq + hq] = Ltot * kLn2;
     counters[(size_t)b * g.Hq + hq] = 0;
   }
-  if (split_lse)
-    for (int i = tid; i <= ns; i += blockDim.x) {
-      const float* pj = base + (size_t)i * (D + 2);
-      const float l = __ldcg(pj + D + 1);
-      split_lse[((size_t)b * g.Hq + hq) * (ns + 1) + i] = l > 0.f ? (__ldcg(pj + D) + log2f(l)) * kLn2 : -INFINITY;
-    }
+  if (split_lse) {
+    float* sl = split_lse + ((size_t)b * g.Hq + hq) * (ns + 1);
+    for (int i = tid; i < ns; i += kThr) sl[i] = pl2[2 * i] * kLn2;
+    // the bf16 partial is the logsumexp of the CTAs' shares
+    const float bl = tid < ns ? pl2[2 * tid + 1] : -INFINITY;
+    const float Bm = block_reduce<true>(bl, red);
+    const float Bs = block_reduce<false>(Bm != -INFINITY && bl != -INFINITY ? exp2f(bl - Bm) : 0.f, red);
+    if (tid == 0) sl[ns] = Bm == -INFINITY ? -INFINITY : (Bm + log2f(Bs)) * kLn2;
+  }
 }
 
 template <int D, int C>
@@ -644,23 +861,17 @@ static cudaError_t decode_as(const Geo& g, int layer, int step, int batch, const
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < kMaxDevices) attr_set[dev] = true;
   }
-  dim3 grid(ns + 1, g.Hq, batch);
+  dim3 grid(ns, g.Hq, batch);
   decode_kernel<D, C><<<grid, kThr, Dec<D, C>::SMEM, s>>>(g, layer, step, q, ctx_len, coded_len, sink, ring, idx,
                                                           cbp, rope, ns, ws, out, lse, split_lse, st);
   return cudaGetLastError();
 }
 
-// Sink + recent-window slots the bf16-partial CTA can stage: K and V rows, the
-// fine RoPE rows and the coarse rows its positions need must fit in its
-// shared memory, and its 4-thread-per-token scoring covers at most 4 passes.
+// Sink + recent-window tokens one call can take: a CTA keeps the scores of its
+// share of them in its score array (num_splits = 1 gives one CTA all of them).
 template <int D, int C>
 static int bf16_capacity_as() {
-  const int F = D / 2;
-  // bytes: 4*D per token (K and V), 8*F*8 fine rows, (tokens/8 + 3) coarse rows of 8*F
-  const int avail = Dec<D, C>::OFF_PW - 8 * F * 8 - 3 * 8 * F;
-  const int by_smem = avail / (4 * D + F);
-  const int by_passes = 4 * (kThr / 4);
-  return by_smem < by_passes ? by_smem : by_passes;
+  return Dec<D, C>::NSC;
 }
 
 int decode_bf16_capacity(int d, int c) {

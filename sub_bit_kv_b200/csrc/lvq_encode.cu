@@ -60,8 +60,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_prefill_kernel(
     if (acc < best) { best = acc; bk = k; }
   }
   const int cn = coded_offset + local;
-  uint8_t* page = idx + idx_page_off(g, layer, blk, req, h, cn >> 3);
-  page[kvi * g.ng * kPage + grp * kPage + (cn & 7)] = (uint8_t)bk;
+  idx[idx_code_off(g, layer, blk, req, h, kvi, cn, grp)] = (uint8_t)bk;
 }
 
 template <int G, int C>
@@ -223,8 +222,7 @@ __global__ void __launch_bounds__(kPageThreads, 2) encode_page_kernel(
       code = bk;
     }
     if (lane == 0) {
-      uint8_t* page = idx + idx_page_off(g, layer, blk, b, h, cn >> 3);
-      page[kvi * g.ng * kPage + grp * kPage + (cn & 7)] = (uint8_t)code;
+      idx[idx_code_off(g, layer, blk, b, h, kvi, cn, grp)] = (uint8_t)code;
     }
   }
 }

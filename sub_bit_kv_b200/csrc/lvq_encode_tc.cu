@@ -349,8 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
         tc_fence_before();
         if (valid_row && ok) {
           const int cn = coded_offset + (t0 + row - tok_begin);
-          uint8_t* page = idx + idx_page_off(g, layer, blk, req, h, cn >> 3);
-          page[kvi * g.ng * kPage + (span * NGC + gi) * kPage + (cn & 7)] = (uint8_t)code;
+          idx[idx_code_off(g, layer, blk, req, h, kvi, cn, span * NGC + gi)] = (uint8_t)code;
         }
         named_sync(1 + set, kRows);     // the set's TMEM columns and A tile are free again
         mma_phase ^= 1u;                // one completed phase of this set's barrier per group

@@ -71,8 +71,7 @@ __global__ void dequant_kernel(Geo g, int layer, int step, int req, int kv, cons
     int h = (int)((i / g.d) % g.H);
     int n = tok_begin + (int)(i / ((size_t)g.d * g.H));
     int grp = ch / g.c, e = ch % g.c;
-    const uint8_t* page = idx + idx_page_off(g, layer, blk, req, h, n >> 3);
-    int code = page[kv * g.ng * kPage + grp * kPage + (n & 7)];
+    const int code = idx[idx_code_off(g, layer, blk, req, h, kv, n, grp)];
     const __nv_bfloat16* slice = cbp + cbp_slice_off(g, layer, kv, blk, h, s);
     out[i] = slice[((size_t)code * g.ng + grp) * g.c + e];
   }

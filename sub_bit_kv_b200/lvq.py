@@ -236,7 +236,7 @@ class CodedCache:
 
     def idx_view(self):
         c, l = self.cfg, self.lay
-        return self.idx.view(c.n_layers, l.n_blocks, c.max_batch, c.n_kv_heads, l.max_pages, 2, l.n_groups, 8)
+        return self.idx.view(c.n_layers, l.n_blocks, c.max_batch, c.n_kv_heads, 2, l.max_pages, l.n_groups, 8)
 
     def check_status(self, where="device"):
         s = int(self.status.item())

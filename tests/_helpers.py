@@ -33,17 +33,17 @@ def make_cfg(w: synth.Workload, n_layers=None, max_batch=None, max_ctx=None, max
 def put_codes(cache: lvq.CodedCache, layer: int, b: int, kv: int, codes: torch.Tensor, offset: int = 0):
     """codes: uint8 [n_blk][N][H][n_g] (logical) -> coded slots offset..offset+N of request b."""
     n_blk, N, H, ng = codes.shape
-    view = cache.idx_view()                               # [L][n_blk][B][H][P][2][n_g][8]
-    flat = view[layer, :, b, :, :, kv]                    # [n_blk][H][P][n_g][8]
+    view = cache.idx_view()                               # [L][n_blk][B][H][2][P][n_g][8]
+    flat = view[layer, :, b, :, kv]                       # [n_blk][H][P][n_g][8]
     flat = flat.permute(0, 1, 2, 4, 3).reshape(n_blk, H, -1, ng)   # [n_blk][H][P*8][n_g]
     flat[:, :, offset:offset + N, :] = codes.permute(0, 2, 1, 3).to(flat.device)
-    view[layer, :, b, :, :, kv] = flat.reshape(n_blk, H, -1, 8, ng).permute(0, 1, 2, 4, 3)
+    view[layer, :, b, :, kv] = flat.reshape(n_blk, H, -1, 8, ng).permute(0, 1, 2, 4, 3)
 
 
 def get_codes(cache: lvq.CodedCache, layer: int, b: int, kv: int, offset: int, N: int) -> torch.Tensor:
     """Inverse of put_codes: uint8 [n_blk][N][H][n_g] on the CPU."""
     view = cache.idx_view()
-    flat = view[layer, :, b, :, :, kv]
+    flat = view[layer, :, b, :, kv]
     n_blk, H, P, ng, _ = flat.shape
     flat = flat.permute(0, 1, 2, 4, 3).reshape(n_blk, H, P * 8, ng)
     return flat[:, :, offset:offset + N, :].permute(0, 2, 1, 3).cpu()

@@ -45,7 +45,7 @@ def test_layout_closed_forms(name):
     lay = lvq.lvq_cache_layout(cfg)
     c, ng, nblk = O.geometry(w.head_dim, w.T, w.Tc, w.G)
     assert (lay.c, lay.n_groups, lay.n_blocks) == (c, ng, nblk)
-    assert lay.page_bytes == 2 * ng * 8
+    assert lay.page_bytes == ng * 8
     assert lay.ring_tokens == w.n_recent + 8
     # code bytes per token, head and K/V: one row of n_g bytes per block ("one index row per Tc block")
     per_token = lay.idx_bytes / (cfg.n_layers * cfg.max_batch * cfg.n_kv_heads * lay.max_pages * 8 * 2)

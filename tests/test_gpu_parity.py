@@ -160,6 +160,17 @@ def test_decode_gqa_two_query_heads_per_kv_head():
     _check_decode(case, 0, 1, q, 4)
 
 
+@pytest.mark.parametrize("ns", [1, 2])
+def test_decode_long_split_several_super_chunks(ns):
+    """A split longer than one CTA's score array (5280 tokens at head_dim 128, c = 4) is
+    processed as several super-chunks, each with its own maximum and fixed-point scale."""
+    w = _reduced("ouro14_g16_32k", n_layers=1, n_kv_heads=2, n_q_heads=2)
+    case = Hl.build_case(w, layers=1, ctx=[4 + 12000 + 128], max_splits=4)
+    for step in (0, 3):
+        q = synth.queries(w, 0, step).cuda()
+        _check_decode(case, 0, step, q, ns)
+
+
 def test_split_count_sweep_agrees():
     w = _reduced("ouro14_g16_32k", n_layers=1, n_kv_heads=2, n_q_heads=2)
     case = Hl.build_case(w, layers=1, ctx=[4000])
@@ -204,7 +215,7 @@ def test_identical_codes_zero_key_share_uniform_attention():
     step = 1
     c.cb_view()[0, 0, :, :, :, 42, step * w.c:(step + 1) * w.c] = 0
     lvq.lvq_pack_codebooks(case.cfg, c.lay, c.cb, c.cbp)
-    c.idx.view(c.idx_view().shape)[..., 0, :, :] = 42       # every K code -> 42
+    c.idx.view(c.idx_view().shape)[:, :, :, :, 0] = 42      # every K code -> 42
     c.sink_view()[:, 0].zero_()
     c.ring_view()[:, 0].zero_()
     q = synth.queries(w, 0, step).cuda()
@@ -250,13 +261,14 @@ def test_page_encode_matches_oracle_and_advances():
     after = c.idx.view(c.idx_view().shape)
     b4 = before.view(c.idx_view().shape)
     assert torch.equal(after[:, :, 1], b4[:, :, 1])
-    assert torch.equal(after[:, :, 0, :, :12], b4[:, :, 0, :, :12])
+    assert torch.equal(after[:, :, 0, :, :, :12], b4[:, :, 0, :, :, :12])
 
 
-def test_decode_guard_fallback_large_scores():
-    """Keys of one entry are scaled by 100 and used only outside each warp's first page: later
-    scores exceed the split's reference maximum by far more than 2^64, which forces the exact
-    recomputation path.  The result must still match the oracle."""
+def test_decode_large_score_range():
+    """Keys of one entry are scaled by 100 and used only outside the first page of every
+    4-page run: scores then spread far beyond the exponent range of a float weight, most
+    weights underflow to zero against the exact maximum, and the result must still match
+    the oracle."""
     w = synth.WORKLOADS["tiny"]
     case = Hl.build_case(w, layers=1, ctx=[512])
     c = case.cache
