@@ -29,6 +29,7 @@ cpu_baseline / --impl reference: the fp64 oracle timed on a bounded sample
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -57,6 +58,20 @@ def parse():
     ap.add_argument("--profile", default="", choices=["", "decode", "encode"],
                     help="build the workload, run 3 launches of one kernel and exit (for ncu captures)")
     return ap.parse_args()
+
+
+# DRAM bytes (read + write) of one decode_kernel<128,4> launch of this workload, from one ncu
+# capture (`python bench.py --profile decode` under ncu), valid only for the decode source it was
+# taken on: the bench reports it when the file's hash still matches, else null.
+DECODE_TRAFFIC = {"source_sha256": "7fb4269e752830ea83cd013c7ecd68a7fcdf147e1eb3db1025a18720edc55ed0",
+                  "bytes_per_launch": 36761088}
+
+
+def decode_traffic():
+    src = os.path.join(ROOT, "sub_bit_kv_b200", "csrc", "lvq_decode.cu")
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    return DECODE_TRAFFIC["bytes_per_launch"] if sha == DECODE_TRAFFIC["source_sha256"] else None
 
 
 def peaks():
@@ -433,7 +448,7 @@ def gpu_arm(args):
                    "num_splits": ns, "tokens_per_step": TOKENS_PER_STEP,
                    "l2": "inputs larger than L2 (3.5 GB of codes per token)", "parallelism": f"replicas{world}"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": None, "kernel": "decode_kernel<128,4>",
+                     "frac": achieved / hbm_peak, "traffic": decode_traffic(), "kernel": "decode_kernel<128,4>",
                      "peak_kind": peak_kind, "bytes_per_launch": bpl, "launch_ms": per_call_ms},
         "code_stream_GBps": code_stream,
         "cpu_baseline": cb,
