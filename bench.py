@@ -205,7 +205,7 @@ def build_cache(w, lvq, synth, torch, extra_tokens: int, device, request_seed: i
                            scales=sc)
         sv[layer, :, :, 0] = sk.permute(0, 1, 3, 2, 4)
         rv[layer, :, :, 0] = rk.permute(0, 1, 3, 2, 4)
-    lvq.lvq_pack_codebooks(cfg, lay, cache.cb, cache.cbp)
+    lvq.lvq_pack_codebooks(cfg, lay, cache.cb, cache.cbp, cache.cb_norm)
     lvq.lvq_rope_table(cfg, lay, cache.rope)
     for layer in range(w.n_layers):
         kv = synth.loop_kv(w, layer, L, stream="coded", request=request_seed, device=device)
@@ -320,8 +320,8 @@ def gpu_arm(args):
                                              cache.coded_len, cache.sink, cache.ring, cache.idx, cache.cbp,
                                              cache.rope, ns, cache.workspace, out_all[tok, t, layer],
                                              lse_all[tok, t, layer], cache.status, stream=stream)
-        lvq.lvq_encode_page(cfg, lay, B, cache.ctx_len, cache.coded_len, cache.ring, cache.cb, cache.idx,
-                            cache.status, stream=stream)
+        lvq.lvq_encode_page(cfg, lay, B, cache.ctx_len, cache.coded_len, cache.ring, cache.cb, cache.cb_norm,
+                            cache.idx, cache.status, stream=stream)
 
     launches_per_step = TOKENS_PER_STEP * NL + 2
     stream = torch.cuda.Stream(device)

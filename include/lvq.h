@@ -184,10 +184,15 @@ LVQ_API lvq_status lvq_encode_prefill(const lvq_config* cfg, const lvq_layout* l
  * block, head, group) into coded slots coded_len[b] .. coded_len[b] + 7, then
  * advances coded_len[b] by 8.  Requests with fewer recent tokens are left
  * untouched, so the call can be issued every 8 tokens from a CUDA graph.
- *   ctx_len, coded_len: device int32 [batch].  ring: bf16 recent window. */
+ *   ctx_len, coded_len: device int32 [batch] (batch <= 1024, else
+ *     LVQ_EUNSUPPORTED).  ring: bf16 recent window.  cb: logical codebooks.
+ *   cb_norm: their fp32 squared entry norms as lvq_pack_codebooks writes them
+ *     (required).
+ * Every codebook is read once per call whatever the number of due requests. */
 LVQ_API lvq_status lvq_encode_page(const lvq_config* cfg, const lvq_layout* lay, int32_t batch,
                            const int32_t* ctx_len, int32_t* coded_len, const void* ring,
-                           const void* cb, uint8_t* idx, int32_t* dev_status, void* stream);
+                           const void* cb, const float* cb_norm, uint8_t* idx, int32_t* dev_status,
+                           void* stream);
 
 /* Decode attention of loop step `step` of layer `layer` ("LoopVQ summary",
  * "premises and limits"; "LoopVQ article", "when LoopVQ changes the deployment

@@ -174,18 +174,19 @@ lvq_status lvq_encode_prefill(const lvq_config* cfg, const lvq_layout* lay, int3
 }
 
 lvq_status lvq_encode_page(const lvq_config* cfg, const lvq_layout* lay, int32_t batch, const int32_t* ctx_len,
-                           int32_t* coded_len, const void* ring, const void* cb, uint8_t* idx,
-                           int32_t* dev_status, void* stream) {
+                           int32_t* coded_len, const void* ring, const void* cb, const float* cb_norm,
+                           uint8_t* idx, int32_t* dev_status, void* stream) {
   Geo g;
   lvq_status s = check_all(cfg, lay, &g);
   if (s != LVQ_OK) return s;
   if (batch < 0 || batch > g.B) return LVQ_EINVAL;
-  if (batch > 0 && (!ctx_len || !coded_len || !ring || !cb || !idx || !aligned16(ring) || !aligned16(cb) ||
-                    !aligned16(idx)))
+  if (batch > kPageMaxBatch) return LVQ_EUNSUPPORTED;
+  if (batch > 0 && (!ctx_len || !coded_len || !ring || !cb || !cb_norm || !idx || !aligned16(ring) ||
+                    !aligned16(cb) || !aligned16(cb_norm) || !aligned16(idx)))
     return LVQ_EINVAL;
   if ((s = check_device()) != LVQ_OK) return s;
   return cuda_status(launch_encode_page(g, batch, ctx_len, coded_len, static_cast<const __nv_bfloat16*>(ring),
-                                        static_cast<const __nv_bfloat16*>(cb), idx, dev_status,
+                                        static_cast<const __nv_bfloat16*>(cb), cb_norm, idx, dev_status,
                                         static_cast<cudaStream_t>(stream)));
 }
 

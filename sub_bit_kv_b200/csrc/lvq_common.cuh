@@ -93,6 +93,12 @@ __device__ inline void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, u
       :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
 
+// Orders this thread's generic-proxy accesses of shared memory before later
+// async-proxy (bulk copy) writes to it.
+__device__ inline void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ inline uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -115,8 +121,9 @@ cudaError_t launch_encode_prefill(const Geo& g, int layer, int req, const __nv_b
                                   int coded_offset, const __nv_bfloat16* cb, uint8_t* idx,
                                   int32_t* st, cudaStream_t s);
 cudaError_t launch_encode_page(const Geo& g, int batch, const int32_t* ctx_len, int32_t* coded_len,
-                               const __nv_bfloat16* ring, const __nv_bfloat16* cb, uint8_t* idx,
-                               int32_t* st, cudaStream_t s);
+                               const __nv_bfloat16* ring, const __nv_bfloat16* cb, const float* cb_norm,
+                               uint8_t* idx, int32_t* st, cudaStream_t s);
+constexpr int kPageMaxBatch = 1024;     // requests one lvq_encode_page call can take
 cudaError_t launch_decode(const Geo& g, int layer, int step, int batch, const __nv_bfloat16* q,
                           const int32_t* ctx_len, const int32_t* coded_len,
                           const __nv_bfloat16* sink, const __nv_bfloat16* ring, const uint8_t* idx,

@@ -335,10 +335,6 @@ __device__ inline bool mbar_test(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-__device__ inline void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // This CTA's share of the bf16 tokens (list entries j, j + ns, ... of [sink tokens,
 // recent tokens]), computed by one warp.  Per batch of up to 60 tokens the key and
 // value rows and the coarse RoPE rows of their positions, plus (once) the fine RoPE
@@ -373,7 +369,7 @@ __device__ bool bf16_share(Service& service, const Geo& g, int layer, int step, 
   int batch = 0;
   for (int k0 = 0; k0 < nbj && !to; k0 += BB, ++batch) {
     const int nbb = min(BB, nbj - k0);
-    if (batch > 0) fence_proxy_async();          // this warp's reads of the area precede the new copies
+    if (batch > 0) fence_proxy_async_shared();          // this warp's reads of the area precede the new copies
     if (lane == 0) {
       mbar_expect_tx(bar, (batch == 0 ? 8 * F * 8 : 0) + nbb * (F * 8 + 4 * D));
       misc[4] = batch + 1;
@@ -443,7 +439,7 @@ __device__ bool bf16_share(Service& service, const Geo& g, int layer, int step, 
     m = m_new;
     service();
   }
-  fence_proxy_async();                           // the value slice is copied into the area next
+  fence_proxy_async_shared();                           // the value slice is copied into the area next
   __syncwarp();
 #pragma unroll
   for (int u = 0; u < CPL; ++u) part[lane + 32 * u] = to ? 0.f : o[u];

@@ -106,124 +106,257 @@ __device__ inline int page_due(const Geo& g, int ctx, int coded) {
   return 1;
 }
 
-// One CTA per codebook (layer, kv, blk, h, grp), looping over the requests whose
-// page is due, so each codebook is read from memory once.  The codebook and
-// its squared norms sit in shared memory; warp t takes token t of the page and
-// lane l the entries l, l + 32, ...  Distances are first taken in the fp32
-// expansion form n_k - 2 x.C_k; every entry within
-// eps = 2^-14 (||x||^2 + max_k n_k) of the minimum is a candidate (the fp32
-// error is far below eps), and when there are several the candidates are
-// rescored exactly in the fp64 direct form, lowest index on ties.
-constexpr int kPageThreads = 32 * kPage;
+// Page encode.  A codebook's contraction with one page is small -- 8 vectors
+// (the page's tokens) x 256 entries x G -- and every page encode touches every
+// codebook of every layer (201 MB of bf16 at the Ouro-1.4B shapes), so the
+// kernel is built to stream codebooks: a persistent grid whose warps each walk
+// a strided list of codebooks, every codebook (and its fp32 norms) bulk-copied
+// into a 3-deep ring private to the warp, and one tensor-core MMA
+// (mma.sync m16n8k16, bf16 in, fp32 accumulate) per 16 entries x 8 vectors x
+// 16 dimensions, with the page's 8 tokens as the N = 8 columns.  For every
+// request whose page is due the warp then takes the fp32 expansion form
+// n_k - 2 x.C_k; every entry within eps = 2^-14 (||x||^2 + max_k n_k) of the
+// minimum is a candidate (the fp32 error is far below eps), and when there are
+// several they are rescored exactly in the fp64 direct form, lowest index on
+// ties.
+template <int G, int C>
+struct PageEnc {
+  static constexpr int TC = G / C;
+  static constexpr int NW = G == 16 ? 8 : 4;          // warps per CTA
+  static constexpr int NBUF = 3;                      // codebooks in flight per warp
+  static constexpr int CBB = kEntries * G * 2;        // one codebook, bf16
+  static constexpr int NB = kEntries * 4;             // its fp32 squared norms
+  static constexpr int BUF = CBB + NB;
+  static constexpr int KS = G / 16;                   // MMA k-steps
+  static constexpr int MAXB = kPageMaxBatch;
+  static constexpr int OFF_BAR = NW * NBUF * BUF;
+  static constexpr int OFF_DUE = OFF_BAR + NW * NBUF * 8;
+  static constexpr int SMEM = OFF_DUE + 2 * MAXB * 4 + 16;
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+  static_assert(BUF % 16 == 0 && OFF_BAR % 8 == 0, "alignment");
+};
+
+__device__ inline void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ inline void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
 
 template <int G, int C>
-__global__ void __launch_bounds__(kPageThreads, 2) encode_page_kernel(
+__global__ void __launch_bounds__(PageEnc<G, C>::NW * 32, 1) encode_page_kernel(
     Geo g, int batch, const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ coded_len,
-    const __nv_bfloat16* __restrict__ ring, const __nv_bfloat16* __restrict__ cb, uint8_t* __restrict__ idx,
-    int32_t* st) {
-  constexpr int TC = G / C;
-  __shared__ float cbs[kEntries * G];     // fp32 copies of the bf16 entries (exact)
-  __shared__ float nrm[kEntries];
-  __shared__ float nmax_s;
-  long cid = blockIdx.x;
-  const int grp = (int)(cid % g.ng); cid /= g.ng;
-  const int h = (int)(cid % g.H); cid /= g.H;
-  const int blk = (int)(cid % g.nblk); cid /= g.nblk;
-  const int kvi = (int)(cid % 2); cid /= 2;
-  const int layer = (int)cid;
-  const int tid = threadIdx.x, lane = tid & 31, t = tid >> 5;
+    const __nv_bfloat16* __restrict__ ring, const __nv_bfloat16* __restrict__ cb,
+    const float* __restrict__ cb_norm, uint8_t* __restrict__ idx, int32_t* st) {
+  using X = PageEnc<G, C>;
+  constexpr int TC = X::TC, NW = X::NW, NBUF = X::NBUF, KS = X::KS;
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + X::OFF_BAR);
+  int* due = reinterpret_cast<int*>(smem + X::OFF_DUE);     // [n_due] requests, then [n_due] coded_len
+  int* n_due_s = due + 2 * X::MAXB;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  bool any = false;
-  for (int b = 0; b < batch; ++b) any |= page_due(g, ctx_len[b], coded_len[b]) == 1;
-  if (!any) return;
-
-  const __nv_bfloat16* Cg = cb + cb_off(g, layer, kvi, blk, h, grp);
-  for (int i = tid; i < kEntries * G; i += kPageThreads) cbs[i] = __bfloat162float(Cg[i]);
-  if (tid == 0) nmax_s = 0.f;
-  __syncthreads();
-  {
-    const int k = tid;                    // kPageThreads == kEntries
-    double n = 0.0;
-#pragma unroll
-    for (int j = 0; j < G; ++j) n += (double)cbs[k * G + j] * (double)cbs[k * G + j];
-    nrm[k] = (float)n;
-    atomicMax(reinterpret_cast<int*>(&nmax_s), __float_as_int((float)n));
+  if (tid == 0) {
+    int n = 0;
+    for (int b = 0; b < batch; ++b) {
+      const int d = page_due(g, ctx_len[b], coded_len[b]);
+      if (d < 0 && blockIdx.x == 0) set_status(st, LVQ_ECAPACITY);
+      if (d == 1) {
+        due[n] = b;
+        due[X::MAXB + n] = coded_len[b];
+        ++n;
+      }
+    }
+    *n_due_s = n;
+    for (int i = 0; i < NW * NBUF; ++i) mbar_init(smem_addr(&bars[i]), 1);
+    fence_mbar_init();
   }
   __syncthreads();
+  const int n_due = *n_due_s;
+  if (n_due == 0) return;
 
-  for (int b = 0; b < batch; ++b) {
-    const int ctx = ctx_len[b], coded = coded_len[b];
-    const int due = page_due(g, ctx, coded);
-    if (due < 0) {
-      if (blockIdx.x == 0 && tid == 0) set_status(st, LVQ_ECAPACITY);
-      continue;
-    }
-    if (due == 0) continue;
-    const int cn = coded + t;             // this warp's token, coded slot cn
-    const int slot = cn % g.R;            // position S + cn lives in slot (cn mod R)
-    float x[G];
-    float xx = 0.f;
-#pragma unroll
-    for (int s2 = 0; s2 < TC; ++s2) {
-      const __nv_bfloat16* p = ring + ring_off(g, layer, kvi, blk * TC + s2, b, h, slot) + grp * C;
-#pragma unroll
-      for (int e = 0; e < C; ++e) {
-        x[s2 * C + e] = __bfloat162float(p[e]);
-        xx = fmaf(x[s2 * C + e], x[s2 * C + e], xx);
+  const long n_cb = (long)g.L * 2 * g.nblk * g.H * g.ng;   // codebooks, (layer, kv, blk, h, grp) order
+  const long stride = (long)gridDim.x * NW;
+  const long first = (long)blockIdx.x * NW + warp;
+  unsigned char* wbuf = smem + (size_t)warp * NBUF * X::BUF;
+  uint64_t* wbar = bars + warp * NBUF;
+
+  auto issue = [&](long c, int slot) {            // lane 0: codebook c into ring slot `slot`
+    const uint32_t bar = smem_addr(&wbar[slot]);
+    mbar_expect_tx(bar, X::BUF);
+    bulk_g2s(smem_addr(wbuf + slot * X::BUF), cb + (size_t)c * kEntries * G, X::CBB, bar);
+    bulk_g2s(smem_addr(wbuf + slot * X::BUF + X::CBB), cb_norm + (size_t)c * kEntries, X::NB, bar);
+  };
+  if (lane == 0)
+    for (int i = 0; i < NBUF - 1; ++i)
+      if (first + i * stride < n_cb) issue(first + i * stride, i);
+
+  const int q = lane & 3, r8 = lane >> 2;          // C fragment: vectors 2q, 2q+1; entries r8 (+8) of each 16
+  for (long it = 0;; ++it) {
+    const long c = first + it * stride;
+    if (c >= n_cb) break;
+    const int slot = (int)(it % NBUF);
+    if (lane == 0 && c + (NBUF - 1) * stride < n_cb) issue(c + (NBUF - 1) * stride, (int)((it + NBUF - 1) % NBUF));
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_addr(&wbar[slot]), (uint32_t)((it / NBUF) & 1), kWaitIters));
+    if (!ok) {
+      if (lane == 0) {
+        set_status(st, LVQ_ETIMEOUT);
+        for (long j = it; j < it + NBUF && first + j * stride < n_cb; ++j)   // copies still in flight
+          mbar_wait(smem_addr(&wbar[j % NBUF]), (uint32_t)((j / NBUF) & 1), kWaitIters);
       }
+      break;
     }
-    float dv[kEntries / 32];
-    float best = INFINITY;
+    const unsigned char* cbs = wbuf + slot * X::BUF;
+    const float* nrm = reinterpret_cast<const float*>(cbs + X::CBB);
+    long cc = c;
+    const int grp = (int)(cc % g.ng); cc /= g.ng;
+    const int h = (int)(cc % g.H); cc /= g.H;
+    const int blk = (int)(cc % g.nblk); cc /= g.nblk;
+    const int kvi = (int)(cc % 2);
+    const int layer = (int)(cc / 2);
+
+    // squared norms this lane needs, and their maximum over the codebook
+    float nr[16][2];
+    float nmax = 0.f;
 #pragma unroll
-    for (int i = 0; i < kEntries / 32; ++i) {
-      const float* ce = cbs + (lane + 32 * i) * G;
-      float dot = 0.f;
-#pragma unroll
-      for (int j = 0; j < G; ++j) dot = fmaf(x[j], ce[j], dot);
-      dv[i] = fmaf(-2.f, dot, nrm[lane + 32 * i]);
-      best = fminf(best, dv[i]);
+    for (int m = 0; m < 16; ++m) {
+      nr[m][0] = nrm[16 * m + r8];
+      nr[m][1] = nrm[16 * m + r8 + 8];
+      nmax = fmaxf(nmax, fmaxf(nr[m][0], nr[m][1]));
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) best = fminf(best, __shfl_xor_sync(0xffffffffu, best, o));
-    const float thr = best + ldexpf(xx + nmax_s, -14);
-    int n_cand = 0, k_cand = kEntries;
+    for (int o = 4; o < 32; o <<= 1) nmax = fmaxf(nmax, __shfl_xor_sync(0xffffffffu, nmax, o));
+
+    for (int di = 0; di < n_due; ++di) {
+      const int b = due[di], coded = due[X::MAXB + di];
+      // B fragments: vector n = lane/4 (the page's token n), dimensions 16 ks + 2q (+1) and +8 (+9)
+      const int slot_n = (coded + r8) % g.R;
+      uint32_t bf[KS][2];
+      float xxp = 0.f;
 #pragma unroll
-    for (int i = 0; i < kEntries / 32; ++i)
-      if (dv[i] <= thr) { ++n_cand; k_cand = min(k_cand, lane + 32 * i); }
+      for (int ks = 0; ks < KS; ++ks)
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      n_cand += __shfl_xor_sync(0xffffffffu, n_cand, o);
-      k_cand = min(k_cand, __shfl_xor_sync(0xffffffffu, k_cand, o));
-    }
-    int code = k_cand;
-    if (n_cand > 1) {
-      // near-tie: exact fp64 direct-form distances of the candidates, lowest index on ties
-      double bd = 1e300;
-      int bk = kEntries;
+        for (int hh = 0; hh < 2; ++hh) {
+          const int k = 16 * ks + 2 * q + 8 * hh;
+          const int s2 = k / C, e = k % C;
+          const __nv_bfloat16* p = ring + ring_off(g, layer, kvi, blk * TC + s2, b, h, slot_n) + grp * C + e;
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+          bf[ks][hh] = w;
+          xxp = fmaf(bf16_lo(w), bf16_lo(w), xxp);
+          xxp = fmaf(bf16_hi(w), bf16_hi(w), xxp);
+        }
+      xxp += __shfl_xor_sync(0xffffffffu, xxp, 1);
+      xxp += __shfl_xor_sync(0xffffffffu, xxp, 2);          // ||x_n||^2 in the lanes of vector n
+      const float xx0 = __shfl_sync(0xffffffffu, xxp, 4 * (2 * q));
+      const float xx1 = __shfl_sync(0xffffffffu, xxp, 4 * (2 * q + 1));
+      // d[m][0..3]: entries 16m + r8 (vectors 2q, 2q+1) and 16m + r8 + 8 (vectors 2q, 2q+1)
+      float d[16][4];
+#pragma unroll
+      for (int m = 0; m < 16; ++m) {
+        d[m][0] = d[m][1] = d[m][2] = d[m][3] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          uint32_t a[4];
+          const int mi = lane >> 3, rr = lane & 7;
+          const int entry = 16 * m + (mi & 1) * 8 + rr, col = 16 * ks + (mi >> 1) * 8;
+          ldmatrix_x4(a, smem_addr(cbs + entry * (2 * G) + col * 2));
+          mma_bf16_16816(d[m], a, bf[ks][0], bf[ks][1]);
+        }
+        d[m][0] = fmaf(-2.f, d[m][0], nr[m][0]);
+        d[m][1] = fmaf(-2.f, d[m][1], nr[m][0]);
+        d[m][2] = fmaf(-2.f, d[m][2], nr[m][1]);
+        d[m][3] = fmaf(-2.f, d[m][3], nr[m][1]);
+      }
+      float best0 = INFINITY, best1 = INFINITY;
+#pragma unroll
+      for (int m = 0; m < 16; ++m) {
+        best0 = fminf(best0, fminf(d[m][0], d[m][2]));
+        best1 = fminf(best1, fminf(d[m][1], d[m][3]));
+      }
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        best0 = fminf(best0, __shfl_xor_sync(0xffffffffu, best0, o));
+        best1 = fminf(best1, __shfl_xor_sync(0xffffffffu, best1, o));
+      }
+      const float thr0 = best0 + (xx0 + nmax) * 6.103515625e-05f;   // 2^-14
+      const float thr1 = best1 + (xx1 + nmax) * 6.103515625e-05f;
+      // candidates as bit masks: bit 2m + hh is entry 16m + r8 + 8hh (increasing with the bit)
+      uint32_t mk0 = 0u, mk1 = 0u;
+#pragma unroll
+      for (int m = 0; m < 16; ++m)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          if (d[m][2 * hh] <= thr0) mk0 |= 1u << (2 * m + hh);
+          if (d[m][2 * hh + 1] <= thr1) mk1 |= 1u << (2 * m + hh);
+        }
+      auto entry_of = [&](int bit) { return 16 * (bit >> 1) + r8 + 8 * (bit & 1); };
+      int n0 = __popc(mk0), n1 = __popc(mk1);
+      int k0 = mk0 ? entry_of(__ffs(mk0) - 1) : kEntries;
+      int k1 = mk1 ? entry_of(__ffs(mk1) - 1) : kEntries;
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        n0 += __shfl_xor_sync(0xffffffffu, n0, o);
+        n1 += __shfl_xor_sync(0xffffffffu, n1, o);
+        k0 = min(k0, __shfl_xor_sync(0xffffffffu, k0, o));
+        k1 = min(k1, __shfl_xor_sync(0xffffffffu, k1, o));
+      }
+      if (__any_sync(0xffffffffu, n0 > 1 || n1 > 1)) {
+        // near-tie: exact fp64 direct-form distances of the candidates, lowest index on ties
 #pragma unroll 1
-      for (int i = 0; i < kEntries / 32; ++i) {
-        if (dv[i] <= thr) {
-          const int k = lane + 32 * i;
-          double acc = 0.0;
+        for (int v = 0; v < 2; ++v) {
+          const bool tie = v == 0 ? n0 > 1 : n1 > 1;
+          uint32_t mk = tie ? (v == 0 ? mk0 : mk1) : 0u;
+          double bd = 1e300;
+          int bk = kEntries;
+          if (mk) {
+            double x[G];
+            const int slot_v = (coded + 2 * q + v) % g.R;
 #pragma unroll
-          for (int j = 0; j < G; ++j) {
-            const double df = (double)x[j] - (double)cbs[k * G + j];
-            acc = fma(df, df, acc);
+            for (int k = 0; k < G; ++k) {
+              const int s2 = k / C, e = k % C;
+              x[k] = (double)__bfloat162float(
+                  ring[ring_off(g, layer, kvi, blk * TC + s2, b, h, slot_v) + grp * C + e]);
+            }
+            while (mk) {
+              const int bit = __ffs(mk) - 1;
+              mk &= mk - 1u;
+              const int e = entry_of(bit);
+              const __nv_bfloat16* ce = reinterpret_cast<const __nv_bfloat16*>(cbs) + e * G;
+              double acc = 0.0;
+#pragma unroll
+              for (int k = 0; k < G; ++k) {
+                const double df = x[k] - (double)__bfloat162float(ce[k]);
+                acc = fma(df, df, acc);
+              }
+              if (acc < bd || (acc == bd && e < bk)) { bd = acc; bk = e; }
+            }
           }
-          if (acc < bd) { bd = acc; bk = k; }
+#pragma unroll
+          for (int o = 4; o < 32; o <<= 1) {
+            const double ob = __shfl_xor_sync(0xffffffffu, bd, o);
+            const int ok2 = __shfl_xor_sync(0xffffffffu, bk, o);
+            if (ob < bd || (ob == bd && ok2 < bk)) { bd = ob; bk = ok2; }
+          }
+          if (tie) {
+            if (v == 0) k0 = bk;
+            else k1 = bk;
+          }
         }
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const double ob = __shfl_xor_sync(0xffffffffu, bd, o);
-        const int ok = __shfl_xor_sync(0xffffffffu, bk, o);
-        if (ob < bd || (ob == bd && ok < bk)) { bd = ob; bk = ok; }
+      if (r8 == 0) {                            // this lane's two tokens (coded_len need not be a multiple of 8)
+        const int n = coded + 2 * q;
+        idx[idx_code_off(g, layer, blk, b, h, kvi, n, grp)] = (uint8_t)k0;
+        idx[idx_code_off(g, layer, blk, b, h, kvi, n + 1, grp)] = (uint8_t)k1;
       }
-      code = bk;
     }
-    if (lane == 0) {
-      idx[idx_code_off(g, layer, blk, b, h, kvi, cn, grp)] = (uint8_t)code;
-    }
+    fence_proxy_async_shared();                 // this warp's reads of the slot precede its refill
+    __syncwarp();
   }
 }
 
@@ -236,20 +369,34 @@ __global__ void advance_kernel(Geo g, int batch, const int32_t* __restrict__ ctx
 
 template <int G, int C>
 static cudaError_t encode_page_as(const Geo& g, int batch, const int32_t* ctx_len, int32_t* coded_len,
-                                  const __nv_bfloat16* ring, const __nv_bfloat16* cb, uint8_t* idx, int32_t* st,
-                                  cudaStream_t s) {
-  const long n_cb = (long)g.L * 2 * g.nblk * g.H * g.ng;
-  encode_page_kernel<G, C><<<(unsigned)n_cb, kPageThreads, 0, s>>>(g, batch, ctx_len, coded_len, ring, cb, idx, st);
+                                  const __nv_bfloat16* ring, const __nv_bfloat16* cb, const float* cb_norm,
+                                  uint8_t* idx, int32_t* st, cudaStream_t s) {
+  using X = PageEnc<G, C>;
+  static int n_sm[kMaxDevices] = {};
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    e = cudaFuncSetAttribute(encode_page_kernel<G, C>, cudaFuncAttributeMaxDynamicSharedMemorySize, X::SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&n_sm[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  encode_page_kernel<G, C><<<n_sm[dev], X::NW * 32, X::SMEM, s>>>(g, batch, ctx_len, coded_len, ring, cb, cb_norm,
+                                                                   idx, st);
   return cudaGetLastError();
 }
 
 cudaError_t launch_encode_page(const Geo& g, int batch, const int32_t* ctx_len, int32_t* coded_len,
-                               const __nv_bfloat16* ring, const __nv_bfloat16* cb, uint8_t* idx,
-                               int32_t* st, cudaStream_t s) {
+                               const __nv_bfloat16* ring, const __nv_bfloat16* cb, const float* cb_norm,
+                               uint8_t* idx, int32_t* st, cudaStream_t s) {
   if (batch == 0) return cudaSuccess;
   cudaError_t e = cudaErrorInvalidValue;
 #define LVQ_PG(GG, CC) \
-  if (g.G == GG && g.c == CC) e = encode_page_as<GG, CC>(g, batch, ctx_len, coded_len, ring, cb, idx, st, s);
+  if (g.G == GG && g.c == CC) e = encode_page_as<GG, CC>(g, batch, ctx_len, coded_len, ring, cb, cb_norm, idx, st, s);
   LVQ_PG(16, 4) LVQ_PG(16, 8) LVQ_PG(16, 16) LVQ_PG(32, 4) LVQ_PG(32, 8) LVQ_PG(32, 16)
 #undef LVQ_PG
   if (e != cudaSuccess) return e;

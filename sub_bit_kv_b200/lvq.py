@@ -52,7 +52,7 @@ _SIGS = {
     "lvq_encode_prefill": [ctypes.POINTER(lvq_config), ctypes.POINTER(lvq_layout), _I32, _I32, _P,
                            ctypes.c_int64, _I32, _I32, _I32, _I32, _P, _P, _P, _P],
     "lvq_encode_page": [ctypes.POINTER(lvq_config), ctypes.POINTER(lvq_layout), _I32, _P, _P, _P, _P, _P,
-                        _P, _P],
+                        _P, _P, _P],
     "lvq_decode_attention": [ctypes.POINTER(lvq_config), ctypes.POINTER(lvq_layout), _I32, _I32, _I32, _P,
                              _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P, _P, _P],
     "lvq_dequantize": [ctypes.POINTER(lvq_config), ctypes.POINTER(lvq_layout), _I32, _I32, _I32, _I32, _P,
@@ -152,11 +152,12 @@ def lvq_encode_prefill(cfg, lay, layer, req, kv, tok_begin, n_tok, coded_offset,
         _stream(stream)), "lvq_encode_prefill")
 
 
-def lvq_encode_page(cfg, lay, batch, ctx_len, coded_len, ring, cb, idx, dev_status, stream=None):
+def lvq_encode_page(cfg, lay, batch, ctx_len, coded_len, ring, cb, cb_norm, idx, dev_status, stream=None):
     _check(lib().lvq_encode_page(
         ctypes.byref(cfg), ctypes.byref(lay), batch, _ptr(ctx_len, "ctx_len", torch.int32, 4 * batch),
         _ptr(coded_len, "coded_len", torch.int32, 4 * batch), _ptr(ring, "ring", torch.bfloat16, lay.ring_bytes),
-        _ptr(cb, "cb", torch.bfloat16, lay.cb_bytes), _ptr(idx, "idx", torch.uint8, lay.idx_bytes),
+        _ptr(cb, "cb", torch.bfloat16, lay.cb_bytes), _ptr(cb_norm, "cb_norm", torch.float32, lay.cb_norm_bytes),
+        _ptr(idx, "idx", torch.uint8, lay.idx_bytes),
         _ptr(dev_status, "dev_status", torch.int32, 4), _stream(stream)), "lvq_encode_page")
 
 
@@ -213,6 +214,7 @@ class CodedCache:
         self.idx = torch.zeros(lay.idx_bytes, dtype=torch.uint8, device=dev)
         self.cb = torch.zeros(lay.cb_bytes // 2, dtype=torch.bfloat16, device=dev)
         self.cbp = torch.zeros(lay.cbp_bytes // 2, dtype=torch.bfloat16, device=dev)
+        self.cb_norm = torch.zeros(lay.cb_norm_bytes // 4, dtype=torch.float32, device=dev)
         self.sink = torch.zeros(lay.sink_bytes // 2, dtype=torch.bfloat16, device=dev)
         self.ring = torch.zeros(lay.ring_bytes // 2, dtype=torch.bfloat16, device=dev)
         self.rope = torch.zeros(lay.rope_bytes // 4, dtype=torch.float32, device=dev)

@@ -105,7 +105,7 @@ def build_case(w: synth.Workload, layers: int, ctx: list, coded: Optional[list] 
                 put_codes(cache, layer, b, 0, ck.to(device))
                 put_codes(cache, layer, b, 1, cv.to(device))
                 codes[(layer, b)] = (ck, cv)
-    lvq.lvq_pack_codebooks(cfg, lay, cache.cb, cache.cbp)
+    lvq.lvq_pack_codebooks(cfg, lay, cache.cb, cache.cbp, cache.cb_norm)
     lvq.lvq_rope_table(cfg, lay, cache.rope)
     if codes_from == "encode":
         for layer in range(layers):

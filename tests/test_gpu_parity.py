@@ -214,7 +214,7 @@ def test_identical_codes_zero_key_share_uniform_attention():
     c = case.cache
     step = 1
     c.cb_view()[0, 0, :, :, :, 42, step * w.c:(step + 1) * w.c] = 0
-    lvq.lvq_pack_codebooks(case.cfg, c.lay, c.cb, c.cbp)
+    lvq.lvq_pack_codebooks(case.cfg, c.lay, c.cb, c.cbp, c.cb_norm)
     c.idx.view(c.idx_view().shape)[:, :, :, :, 0] = 42      # every K code -> 42
     c.sink_view()[:, 0].zero_()
     c.ring_view()[:, 0].zero_()
@@ -231,37 +231,43 @@ def test_identical_codes_zero_key_share_uniform_attention():
 
 # ----------------------------------------------------------------------------------- page encode
 
-def test_page_encode_matches_oracle_and_advances():
-    w = _reduced("ouro14_tc2_64k", n_layers=2, n_kv_heads=2, n_q_heads=2, n_recent=16)
+@pytest.mark.parametrize("name", ["ouro14_tc2_64k", "ouro14_g16_32k", "ouro14_g32_b32"])
+def test_page_encode_matches_oracle_and_advances(name):
+    """Requests 0 and 2 have a full recent window and are encoded (several due requests share
+    each codebook read); request 1 is one token short and is left untouched."""
+    w = _reduced(name, n_layers=2, n_kv_heads=2, n_q_heads=2, n_recent=16)
     R = w.n_recent + 8
-    # request 0: recent window full (R tokens) -> encoded; request 1: one short -> untouched
-    ctx = [w.n_sink + 100 + R, w.n_sink + 50 + R - 1]
-    case = Hl.build_case(w, layers=2, ctx=ctx, coded=[100, 50])
+    ctx = [w.n_sink + 100 + R, w.n_sink + 50 + R - 1, w.n_sink + 64 + R]
+    case = Hl.build_case(w, layers=2, ctx=ctx, coded=[100, 50, 64])
     c = case.cache
     before = c.idx.clone()
-    lvq.lvq_encode_page(case.cfg, c.lay, 2, c.ctx_len, c.coded_len, c.ring, c.cb, c.idx, c.status)
+    lvq.lvq_encode_page(case.cfg, c.lay, 3, c.ctx_len, c.coded_len, c.ring, c.cb, c.cb_norm, c.idx, c.status)
     torch.cuda.synchronize()
     c.check_status()
-    assert c.coded_len.cpu().tolist() == [108, 50]
-    for layer in range(2):
-        rk = Hl.f64(case.ring_kv[(layer, 0)])                 # [2][T][R][H][d], oldest first
-        ck, cv = O.page_encode(rk[0], rk[1], Hl.f64(case.cb[layer][0]), Hl.f64(case.cb[layer][1]), w.Tc, w.G)
-        got_k = Hl.get_codes(c, layer, 0, 0, 100, 8).numpy()
-        got_v = Hl.get_codes(c, layer, 0, 1, 100, 8).numpy()
-        # compare through the near-tie rule
-        for kvi, (got, ref) in enumerate(((got_k, ck), (got_v, cv))):
-            X = O.joint_vectors(rk[kvi][:, :8], w.Tc, w.G)
-            cbk = Hl.f64(case.cb[layer][kvi])
-            for blk in range(X.shape[0]):
-                for h in range(X.shape[2]):
-                    for g in range(X.shape[3]):
-                        check_codes(got[blk, :, h, g], X[blk, :, h, g], cbk[blk, h, g])
-            assert (got == ref).mean() > 0.999
-    # request 1's codes and request 0's other pages are untouched
+    assert c.coded_len.cpu().tolist() == [108, 50, 72]
+    for b, off in ((0, 100), (2, 64)):
+        for layer in range(2):
+            rk = Hl.f64(case.ring_kv[(layer, b)])                 # [2][T][R][H][d], oldest first
+            ck, cv = O.page_encode(rk[0], rk[1], Hl.f64(case.cb[layer][0]), Hl.f64(case.cb[layer][1]), w.Tc, w.G)
+            got_k = Hl.get_codes(c, layer, b, 0, off, 8).numpy()
+            got_v = Hl.get_codes(c, layer, b, 1, off, 8).numpy()
+            # compare through the near-tie rule
+            for kvi, (got, ref) in enumerate(((got_k, ck), (got_v, cv))):
+                X = O.joint_vectors(rk[kvi][:, :8], w.Tc, w.G)
+                cbk = Hl.f64(case.cb[layer][kvi])
+                for blk in range(X.shape[0]):
+                    for h in range(X.shape[2]):
+                        for g in range(X.shape[3]):
+                            check_codes(got[blk, :, h, g], X[blk, :, h, g], cbk[blk, h, g])
+                assert (got == ref).mean() > 0.999
+    # request 1's codes and the other pages of requests 0 and 2 are untouched
     after = c.idx.view(c.idx_view().shape)
     b4 = before.view(c.idx_view().shape)
     assert torch.equal(after[:, :, 1], b4[:, :, 1])
     assert torch.equal(after[:, :, 0, :, :, :12], b4[:, :, 0, :, :, :12])
+    assert torch.equal(after[:, :, 0, :, :, 14:], b4[:, :, 0, :, :, 14:])
+    assert torch.equal(after[:, :, 2, :, :, :8], b4[:, :, 2, :, :, :8])
+    assert torch.equal(after[:, :, 2, :, :, 9:], b4[:, :, 2, :, :, 9:])
 
 
 def test_decode_large_score_range():
@@ -275,7 +281,7 @@ def test_decode_large_score_range():
     cbv = c.cb_view()
     cbv[0, 0, :, :, :, 7, :] = (cbv[0, 0, :, :, :, 7, :].float() * 100).to(torch.bfloat16)
     case.cb[0][0, :, :, :, 7, :] = cbv[0, 0, :, :, :, 7, :].cpu()
-    lvq.lvq_pack_codebooks(case.cfg, c.lay, c.cb, c.cbp)
+    lvq.lvq_pack_codebooks(case.cfg, c.lay, c.cb, c.cbp, c.cb_norm)
     ck, cv = case.codes[(0, 0)]
     ck = ck.clone()
     n = torch.arange(ck.shape[1])
