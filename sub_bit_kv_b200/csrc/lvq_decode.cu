@@ -65,7 +65,6 @@ struct Dec {
   static constexpr int NP = NG / 2;        // pair-groups (groups g, g + NG/2)
   static constexpr int TQ = 32 / NP;       // token phases of the score mapping
   static constexpr int TPL = kPage / TQ;   // score tokens per lane per page
-  static constexpr int GRP = NP / TPL;     // lanes holding the same reduced score
   static constexpr int TPV = 32 / NG;      // lanes per group in the value phase
   static constexpr int VPL = kPage / TPV;  // value tokens per lane per page
   static constexpr int SH = NG == 32 ? 7 : NG == 16 ? 6 : 5;   // log2 of a histogram row in bytes
@@ -171,7 +170,6 @@ struct Lane {
   int P, tq;
   uint32_t gb_lo, gb_hi;              // byte offsets of the lane's two groups inside a slice row
   uint32_t sel[2];
-  int i_own;                          // index, among the lane's tokens of a page, of the one it ends up holding
   float2 twoc[C], mtwoc[C];           // (2 cos, 2 cos) and its negation, of the lane's token stride
 };
 
@@ -192,83 +190,83 @@ __device__ inline void lane_init(Lane<D, C>& L, int lane, const float* rope, int
     L.twoc[e] = make_float2(2.f * r.x, 2.f * r.x);
     L.mtwoc[e] = make_float2(-2.f * r.x, -2.f * r.x);
   }
-  L.i_own = L.P / X::GRP;
 }
 
-// Scores of the 8 tokens of one page.  On return the lane holds the score of
-// token t_own = tq + TQ * (P / GRP).  With n counting the lane's tokens from the
-// chunk start, the state (Wc, Wn) holds X_n = s_n W_n and X_{n+1}, where
-// s_n = +1, +1, -1, -1, ... (period 4): then X_{n+2} = k X_{n+1} + X_n with
-// k = +2 cos(s theta) for odd n and -2 cos(s theta) for even n -- no negated
-// operand -- and the token's score is s_n times the dot product with X_n.  `ph` is
-// n mod 4 of the page's first token.  With one token per lane per page (TPL = 1)
-// the state is plain W_n and W_{n+2} = 2 cos W_{n+1} - W_n.  The state moves on by
-// TPL tokens.
+// Scores of the warp's kPPW pages of a chunk (kPPW * 8 tokens).  Lane (tq, P)
+// owns pair-group P and, in page pi, the tokens tq + TQ i (i < TPL): n = pi TPL + i
+// counts its NP = kPPW TPL tokens.  It accumulates each token's partial dot
+// product over its pair-group; one transposed reduction over the NP lanes of a
+// token phase then leaves lane (tq, P) with the full score of its own token,
+// n = P: page P / TPL, token tq + TQ (P % TPL).
+// The recurrence state (Wc, Wn) holds X_n = s_n W_n and X_{n+1}, s_n = +1, +1,
+// -1, -1, ... (period 4): X_{n+2} = k X_{n+1} + X_n with k = +2 cos(s theta)
+// for odd n and -2 cos(s theta) for even n -- no negated operand -- and token n
+// scores s_n times the dot product with X_n.  On return the state has moved on by
+// NP tokens.
 template <int D, int C>
-__device__ inline float page_scores(const Lane<D, C>& L, const unsigned char* Ks, const unsigned char* pg,
-                                    float2 (&Wc)[C], float2 (&Wn)[C], int ph) {
+__device__ inline float run_scores(const Lane<D, C>& L, const unsigned char* Ks, const unsigned char* pages,
+                                   float2 (&Wc)[C], float2 (&Wn)[C]) {
   using X = Dec<D, C>;
   constexpr int TQ = X::TQ, TPL = X::TPL, NP = X::NP;
-  const uint2 wlo = *reinterpret_cast<const uint2*>(pg + L.P * kPage);
-  const uint2 whi = *reinterpret_cast<const uint2*>(pg + (L.P + NP) * kPage);
-  float acc[TPL];
+  static_assert(kPPW * TPL == NP, "one token per lane after the reduction");
+  float acc[NP];
 #pragma unroll
-  for (int i = 0; i < TPL; ++i) {
-    uint32_t xl, xh, sel;
-    if constexpr (TQ == 8) {
-      xl = L.tq < 4 ? wlo.x : wlo.y;
-      xh = L.tq < 4 ? whi.x : whi.y;
-      sel = L.sel[0];
-    } else {
-      const int word = (TQ * i) / 4;                 // compile-time
-      xl = word ? wlo.y : wlo.x;
-      xh = word ? whi.y : whi.x;
-      sel = L.sel[(TQ * i / 2) & 1];
-    }
-    uint32_t lo[C / 2], hi[C / 2];
-    load_row<C>(Ks, row_addr<D>(xl, L.gb_lo, sel), lo);
-    load_row<C>(Ks, row_addr<D>(xh, L.gb_hi, sel), hi);
-    float2 a2 = make_float2(0.f, 0.f);
+  for (int pi = 0; pi < kPPW; ++pi) {
+    const unsigned char* pg = pages + pi * X::PAGE;
+    const uint2 wlo = *reinterpret_cast<const uint2*>(pg + L.P * kPage);
+    const uint2 whi = *reinterpret_cast<const uint2*>(pg + (L.P + NP) * kPage);
 #pragma unroll
-    for (int w = 0; w < C / 2; ++w) {
-      a2 = __ffma2_rn(Wc[2 * w], make_float2(bf16_lo(lo[w]), bf16_lo(hi[w])), a2);
-      a2 = __ffma2_rn(Wc[2 * w + 1], make_float2(bf16_hi(lo[w]), bf16_hi(hi[w])), a2);
-    }
-    acc[i] = a2.x + a2.y;
+    for (int i = 0; i < TPL; ++i) {
+      const int n = pi * TPL + i;                    // compile-time
+      uint32_t xl, xh, sel;
+      if constexpr (TQ == 8) {
+        xl = L.tq < 4 ? wlo.x : wlo.y;
+        xh = L.tq < 4 ? whi.x : whi.y;
+        sel = L.sel[0];
+      } else {
+        const int word = (TQ * i) / 4;
+        xl = word ? wlo.y : wlo.x;
+        xh = word ? whi.y : whi.x;
+        sel = L.sel[(TQ * i / 2) & 1];
+      }
+      uint32_t lo[C / 2], hi[C / 2];
+      load_row<C>(Ks, row_addr<D>(xl, L.gb_lo, sel), lo);
+      load_row<C>(Ks, row_addr<D>(xh, L.gb_hi, sel), hi);
+      float2 a2 = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int e = 0; e < C; ++e) {
-      float2 nx;
-      if constexpr (TPL >= 2)       // the page starts at even n: n + i is odd exactly for odd i
-        nx = __ffma2_rn((i & 1) ? L.twoc[e] : L.mtwoc[e], Wn[e], Wc[e]);
-      else
-        nx = __ffma2_rn(L.twoc[e], Wn[e], make_float2(-Wc[e].x, -Wc[e].y));
-      Wc[e] = Wn[e];
-      Wn[e] = nx;
+      for (int w = 0; w < C / 2; ++w) {
+        a2 = __ffma2_rn(Wc[2 * w], make_float2(bf16_lo(lo[w]), bf16_lo(hi[w])), a2);
+        a2 = __ffma2_rn(Wc[2 * w + 1], make_float2(bf16_hi(lo[w]), bf16_hi(hi[w])), a2);
+      }
+      acc[n] = (n & 2) ? -a2.x - a2.y : a2.x + a2.y;
+#pragma unroll
+      for (int e = 0; e < C; ++e) {
+        const float2 nx = __ffma2_rn((n & 1) ? L.twoc[e] : L.mtwoc[e], Wn[e], Wc[e]);
+        Wc[e] = Wn[e];
+        Wn[e] = nx;
+      }
     }
   }
-  // transposed reduction over the NP lanes of a token phase
-  int cnt = TPL;
+  // transposed reduction over the NP lanes of a token phase: at each level a lane
+  // keeps the half of its values selected by bit o of P and adds its partner's
 #pragma unroll
   for (int o = NP / 2; o > 0; o >>= 1) {
-    if (cnt > 1) {
-      const int half = cnt / 2;
-      const bool up = (L.P & o) != 0;
+    const bool up = (L.P & o) != 0;
 #pragma unroll
-      for (int k = 0; k < (TPL > 1 ? TPL / 2 : 1); ++k) {
-        if (k < half) {
-          const float send = up ? acc[k] : acc[k + half];
-          const float keep = up ? acc[k + half] : acc[k];
-          acc[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-        }
-      }
-      cnt = half;
-    } else {
-      acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], o);
+    for (int k = 0; k < o; ++k) {
+      const float send = up ? acc[k] : acc[k + o];
+      const float keep = up ? acc[k + o] : acc[k];
+      acc[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
     }
   }
-  if constexpr (TPL >= 2) return ((ph + L.i_own) & 2) ? -acc[0] : acc[0];
   return acc[0];
 }
+
+// Programmatic dependent launch: wait until the preceding kernel of the stream
+// has completed and its writes are visible; let the next kernel launch early.
+// Without a programmatic predecessor or successor both are no-ops.
+__device__ inline void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ inline void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // Barrier of the compute warps only (the producer warp never joins it).
 __device__ inline void compute_sync() {
@@ -420,8 +418,8 @@ __device__ bool bf16_share(Service& service, const Geo& g, int layer, int step, 
           if (k < 32) sc0 = acc[t];
           else sc1 = acc[t];
         }
+        service();
       }
-      service();
     }
     // online softmax across batches
     const float m_new = fmaxf(m, warp_max(fmaxf(sc0, sc1)));
@@ -435,6 +433,7 @@ __device__ bool bf16_share(Service& service, const Geo& g, int layer, int step, 
       const float pk = __shfl_sync(0xffffffffu, k < 32 ? p0 : p1, k & 31);
 #pragma unroll
       for (int u = 0; u < CPL; ++u) o[u] = fmaf(pk, __bfloat162float(vb[k * D + lane + 32 * u]), o[u]);
+      if ((k & 3) == 3) service();
     }
     m = m_new;
     service();
@@ -459,7 +458,7 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
     float* __restrict__ ws, float* __restrict__ out, float* __restrict__ lse, float* __restrict__ split_lse,
     int32_t* st) {
   using X = Dec<D, C>;
-  constexpr int F = X::F, NG = X::NG, TQ = X::TQ, GRP = X::GRP, NPAIR = X::NPAIR, NREP = X::NREP;
+  constexpr int F = X::F, NG = X::NG, TQ = X::TQ, NPAIR = X::NPAIR, NREP = X::NREP;
   extern __shared__ __align__(1024) unsigned char smem[];
   unsigned char* Ks = smem;
   const unsigned char* Vsm = smem + X::OFF_V;
@@ -485,6 +484,27 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
   float* part_coded = ws + (slot0 + 2 * j) * (D + 2);
   float* part_bf16 = ws + (slot0 + 2 * j + 1) * (D + 2);
   int32_t* counters = reinterpret_cast<int32_t*>(ws + (size_t)g.B * g.Hq * g.max_splits * 2 * (D + 2));
+
+  if (tid == 0) {
+    for (int i = 0; i < X::NBAR; ++i) mbar_init(smem_addr(&bars[i]), i >= 2 + kStages && i < 2 + 2 * kStages ? kCW : 1);
+    fence_mbar_init();
+    misc[0] = 0;
+    misc[1] = 0;
+    misc[2] = 0;
+    misc[3] = 0;
+    misc[4] = 0;
+  }
+  __syncthreads();
+  // The step-t key slice depends on nothing another kernel of a decode sequence writes, so it is
+  // fetched before waiting for the preceding kernel in the stream (programmatic dependent launch):
+  // its latency overlaps that kernel's tail.  Everything else is read after the wait.
+  if (producer && lane == 0) {
+    const uint32_t bk = smem_addr(&bars[0]);
+    mbar_expect_tx(bk, X::KS);
+    bulk_g2s(smem_addr(Ks), cbp + cbp_slice_off(g, layer, 0, blk, h, s), X::KS, bk);
+  }
+  grid_dependency_wait();
+  launch_dependents();
 
   const int ctx = ctx_len[b], Lc = coded_len[b];
   const int S_eff = min(g.S, max(ctx, 0));
@@ -525,26 +545,12 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
              np * X::PAGE, bar);
   };
 
-  if (tid == 0) {
-    for (int i = 0; i < X::NBAR; ++i) mbar_init(smem_addr(&bars[i]), i >= 2 + kStages && i < 2 + 2 * kStages ? kCW : 1);
-    fence_mbar_init();
-    misc[0] = 0;
-    misc[1] = 0;
-    misc[2] = 0;
-    misc[3] = 0;
-    misc[4] = 0;
-  }
-  __syncthreads();
-  // ---- prologue: the producer starts the K slice and the first chunks; compute threads rotate the
-  // query (scaled so that scores come out in log2 units) and clear the histogram
+  // ---- prologue: the producer starts the first chunks; compute threads rotate the query (scaled so
+  // that scores come out in log2 units) and clear the histogram
   const int nb = bad ? 0 : S_eff + recent;                 // bf16 tokens: [sink tokens, recent tokens]
   const int nbj = nb > j ? (nb - j + ns - 1) / ns : 0;    // this CTA's share: j, j + ns, ...
-  if (producer && lane == 0 && do_coded) {
-    const uint32_t bk = smem_addr(&bars[0]);
-    mbar_expect_tx(bk, X::KS);
-    bulk_g2s(smem_addr(Ks), cbp + cbp_slice_off(g, layer, 0, blk, h, s), X::KS, bk);
+  if (producer && lane == 0 && do_coded)
     for (int ci = 0; ci < min(kStages, n_stream); ++ci) issue_chunk(ci);
-  }
   if (!bad && tid < F) {
     const __nv_bfloat16* qv = q + ((size_t)b * g.Hq + hq) * D;
     const float2 qraw = make_float2(__bfloat162float(qv[tid]), __bfloat162float(qv[tid + F]));
@@ -604,8 +610,7 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
         const int f = L.P * C + e;
         U[e] = cmul(zq[f], cconj(rope_at(rope, g.RC, F, p_first, f)));
       }
-      const bool writer = (L.P % GRP) == 0;
-      const int t_own = L.tq + TQ * (L.P / GRP);
+      const int pi_own = L.P / X::TPL, t_own = L.tq + TQ * (L.P % X::TPL);   // the lane's token of a run
       const int gv = lane % NG, tp = lane / NG;
       const uint32_t hl = smem_addr(Hs) + (uint32_t)gv * 4;
       uint32_t* PW = reinterpret_cast<uint32_t*>(SC);
@@ -630,16 +635,12 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
               Wc[e] = U[e];
               Wn[e] = cmul(U[e], etq_s[L.P * C + e]);     // s_1 = +1
             }
-#pragma unroll 2
-            for (int pi = 0; pi < kPPW; ++pi) {
-              const int pl = warp * kPPW + pi;
-              const int tb = c0 + kPage * pl;
-              if (tb >= s1) break;
-              const float sc_ = page_scores<D, C>(L, Ks, stage + pl * X::PAGE, Wc, Wn, (pi * X::TPL) & 3);
-              const float sv = tb + t_own < s1 ? sc_ : -INFINITY;
-              mx = fmaxf(mx, sv);
-              if (writer) SC[tb - s0 + t_own] = sv;
-            }
+            // pages past the split's end hold stale codes: their tokens are masked
+            const float sc_ = run_scores<D, C>(L, Ks, stage + warp * kPPW * X::PAGE, Wc, Wn);
+            const int tok = c0 + kPage * (warp * kPPW + pi_own) + t_own;
+            const float sv = tok < s1 ? sc_ : -INFINITY;
+            mx = fmaxf(mx, sv);
+            SC[tok - s0] = sv;
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_addr(&bars[2 + kStages + ci % kStages]));
           }
@@ -747,13 +748,15 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
   if (!do_coded && producer)
     timed_out = bf16_share<D, C>(no_service, g, layer, step, b, h, j, ns, S_eff, Lc, nbj, sink, ring, rope, zq,
                                  smem + X::OFF_V, smem_addr(&bars[2 + 2 * kStages]), part_bf16, misc);
+  // the key slice copy was issued by every CTA: let it land before the CTA can exit
+  if (tid == 0 && !do_coded && !mbar_wait(smem_addr(&bars[0]), 0, kWaitIters)) timed_out = true;
   if (__syncthreads_or(timed_out)) {
     if (tid == 0) {
       set_status(st, LVQ_ETIMEOUT);
+      mbar_wait(smem_addr(&bars[0]), 0, kWaitIters);
       misc[0] = 1;
       if (do_coded) {   // let every issued copy land before the CTA can exit
         const int issued = max(misc[2], min(kStages, n_stream));
-        mbar_wait(smem_addr(&bars[0]), 0, kWaitIters);
         if (misc[3]) mbar_wait(smem_addr(&bars[1]), 0, kWaitIters);
         for (int ci = max(0, issued - kStages); ci < issued; ++ci)
           mbar_wait(smem_addr(&bars[2 + ci % kStages]), (ci / kStages) & 1, kWaitIters);
@@ -857,10 +860,18 @@ static cudaError_t decode_as(const Geo& g, int layer, int step, int batch, const
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < kMaxDevices) attr_set[dev] = true;
   }
-  dim3 grid(ns, g.Hq, batch);
-  decode_kernel<D, C><<<grid, kThr, Dec<D, C>::SMEM, s>>>(g, layer, step, q, ctx_len, coded_len, sink, ring, idx,
-                                                          cbp, rope, ns, ws, out, lse, split_lse, st);
-  return cudaGetLastError();
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(ns, g.Hq, batch);
+  lc.blockDim = dim3(kThr, 1, 1);
+  lc.dynamicSmemBytes = Dec<D, C>::SMEM;
+  lc.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // may start during the previous kernel
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  return cudaLaunchKernelEx(&lc, decode_kernel<D, C>, g, layer, step, q, ctx_len, coded_len, sink, ring, idx, cbp,
+                            rope, ns, ws, out, lse, split_lse, st);
 }
 
 // Sink + recent-window tokens one call can take: a CTA keeps the scores of its

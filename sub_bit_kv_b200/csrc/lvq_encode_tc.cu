@@ -58,7 +58,8 @@ struct Enc {
   static constexpr int OFF_RAW = OFF_A + NGC * A_TILE;
   static constexpr int OFF_NMAX = OFF_RAW + kRawStages * RAW;
   static constexpr int OFF_BAR = OFF_NMAX + 16 * 4;
-  static constexpr int OFF_TMEM = OFF_BAR + 8 * (kRawStages + 2);
+  static constexpr int OFF_BMIN = OFF_BAR + 8 * (kRawStages + 2);     // [8][256] block minima
+  static constexpr int OFF_TMEM = OFF_BMIN + (kEntries / 32) * kThreads * 4;
   // + alignment slack; at least 120 KB so that one CTA (holding all of TMEM) fits per SM
   static constexpr int SMEM = (OFF_TMEM + 16 + 1024) > 120 * 1024 ? (OFF_TMEM + 16 + 1024) : 120 * 1024;
   static_assert(NGC == 2 || NGC == 4, "two MMA sets alternate over the item's groups");
@@ -122,6 +123,25 @@ __device__ inline void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 64 consecutive fp32 columns of this thread's TMEM lane, issued without waiting
+// (tcgen05.wait::ld completes every load issued before it)
+__device__ inline void tmem_ld64_nowait(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,"
+      "%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr));
+}
+__device__ inline void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
 __device__ inline float fmin3(float a, float b, float c) {
   float d;
   asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -145,6 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + X::OFF_BAR);  // [0..1] raw stages, [2..3] MMA sets
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + X::OFF_TMEM);
   volatile int* fail_s = reinterpret_cast<volatile int*>(smem + X::OFF_TMEM + 4);   // per MMA set
+  float* bmin_s = reinterpret_cast<float*>(smem + X::OFF_BMIN);
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int set = tid / kRows;            // MMA set: warps 0-3 or 4-7
@@ -176,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
   const int n_ranges = (n_tok + kItemTokens - 1) / kItemTokens;
   const long n_items = (long)n_sets * n_ranges;
 
-  uint32_t raw_phase[kRawStages] = {0, 0};
+  uint32_t raw_phase = 0;   // bit s: parity of raw stage s
   uint32_t mma_phase = 0;
   int tile_counter = 0;     // tiles processed by this CTA (drives the raw ring)
   bool failed = false;
@@ -237,11 +258,11 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
     for (int tl = 0; tl < n_tiles && !failed; ++tl, ++tile_counter) {
       const int stg = tile_counter % kRawStages;
       const int t0 = t_first + tl * kTileTokens;
-      if (__syncthreads_or(!mbar_wait(smem_addr(&bars[stg]), raw_phase[stg], kWaitIters))) {
+      if (__syncthreads_or(!mbar_wait(smem_addr(&bars[stg]), (raw_phase >> stg) & 1u, kWaitIters))) {
         failed = true;
         break;
       }
-      raw_phase[stg] ^= 1u;
+      raw_phase ^= 1u << stg;
       const unsigned char* rw = raw + stg * X::RAW;
       const bool valid_row = t0 + row < t_last;
 
@@ -263,13 +284,11 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
           }
 #pragma unroll
         for (int k8 = 0; k8 < G / 8; ++k8) {
-          uint4 w;
-          uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            wp[q] = (uint32_t)__bfloat16_as_ushort(xv[k8 * 8 + 2 * q]) |
-                    ((uint32_t)__bfloat16_as_ushort(xv[k8 * 8 + 2 * q + 1]) << 16);
-          *reinterpret_cast<uint4*>(at + kmaj_off(row, k8 * 8, SBO)) = w;
+          auto pk = [&](int q) {
+            return (uint32_t)__bfloat16_as_ushort(xv[k8 * 8 + 2 * q]) |
+                   ((uint32_t)__bfloat16_as_ushort(xv[k8 * 8 + 2 * q + 1]) << 16);
+          };
+          *reinterpret_cast<uint4*>(at + kmaj_off(row, k8 * 8, SBO)) = make_uint4(pk(0), pk(1), pk(2), pk(3));
         }
         {
           const uint32_t one = 0x3f80u;   // bf16 1.0
@@ -292,56 +311,106 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
         named_sync(1 + set, kRows);
         const bool ok = fail_s[set] == 0;      // uniform over the set
 
-        // epilogue: min of row, then the candidates within eps of it
+        // epilogue: the row's minimum with the minimum of every 32-column block (one wait per 64
+        // columns), then the candidates within eps of it -- only blocks whose minimum is within
+        // eps can hold one, so usually a single block is read again
         const float eps = ldexpf(xx + nmax_s[gi], -14);
-        float m0 = INFINITY, m1 = INFINITY, m2 = INFINITY, m3 = INFINITY;
 #pragma unroll 1
-        for (int q = 0; q < kEntries / 32; ++q) {
-          float v[32];
-          tmem_ld32(tmem_set + lane_addr + q * 32, v);
+        for (int q2 = 0; q2 < kEntries / 64; ++q2) {
+          uint32_t ra[64];
+          tmem_ld64_nowait(tmem_set + lane_addr + q2 * 64, ra);
+          tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            m0 = fmin3(m0, v[i], v[i + 1]);
-            m1 = fmin3(m1, v[i + 2], v[i + 3]);
-            m2 = fmin3(m2, v[i + 4], v[i + 5]);
-            m3 = fmin3(m3, v[i + 6], v[i + 7]);
+          for (int b2 = 0; b2 < 2; ++b2) {
+            const uint32_t* r = ra + 32 * b2;
+            float m0 = __uint_as_float(r[0]), m1 = __uint_as_float(r[1]);
+#pragma unroll
+            for (int i = 2; i < 30; i += 4) {          // columns 2..29
+              m0 = fmin3(m0, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+              m1 = fmin3(m1, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+            }
+            m0 = fmin3(m0, __uint_as_float(r[30]), __uint_as_float(r[31]));
+            bmin_s[(2 * q2 + b2) * kThreads + tid] = fminf(m0, m1);
           }
         }
-        const float thr = fminf(fminf(m0, m1), fminf(m2, m3)) + eps;
-        uint32_t cand = 0;                 // (k+1) of every candidate, 9 bits each, last in the low bits
-#pragma unroll 1
-        for (int q = 0; q < kEntries / 32; ++q) {
-          float v[32];
-          tmem_ld32(tmem_set + lane_addr + q * 32, v);
+        float bmin[kEntries / 32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (v[i] <= thr) cand = (cand << 9) + (uint32_t)(q * 32 + i + 1);
+        for (int q = 0; q < kEntries / 32; ++q) bmin[q] = bmin_s[q * kThreads + tid];
+        float mrow = bmin[0];
+#pragma unroll
+        for (int q = 1; q < kEntries / 32; ++q) mrow = fminf(mrow, bmin[q]);
+        const float thr = mrow + eps;
+        uint32_t bmask = 0;                // blocks that can hold a candidate of this row
+#pragma unroll
+        for (int q = 0; q < kEntries / 32; ++q) bmask |= (bmin[q] <= thr ? 1u : 0u) << q;
+        uint32_t cand = 0;                 // (k+1) of the last 3 candidates, 9 bits each, last in the low bits
+        int n_cand = 0;
+        // the 64-column pairs of blocks any row of the warp needs, in order (tcgen05.ld is
+        // warp-collective); one wait per pair
+        uint32_t pairs = __reduce_or_sync(0xffffffffu, bmask);
+        pairs = (pairs | (pairs >> 1)) & 0x55u;
+        for (; pairs; pairs &= pairs - 1u) {
+          const int q = __ffs(pairs) - 1;           // even: blocks q and q + 1
+          uint32_t r[64];
+          tmem_ld64_nowait(tmem_set + lane_addr + q * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int b2 = 0; b2 < 2; ++b2)
+            if ((bmask >> (q + b2)) & 1u) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (__uint_as_float(r[32 * b2 + i]) <= thr) {
+                  cand = (cand << 9) + (uint32_t)((q + b2) * 32 + i + 1);
+                  ++n_cand;
+                }
+            }
         }
-        int code = (int)cand - 1;
-        const bool tie = cand >= 512u;
+        int code = (int)(cand & 511u) - 1;
+        const bool tie = n_cand > 1;
         if (__any_sync(0xffffffffu, tie && valid_row)) {
-          // near-tie: exact fp64 direct-form distances of the candidates
+          // near-tie: exact fp64 direct-form distances of the candidates, lowest index on ties.
+          // Up to 3 candidates are in `cand`; a row with more rescans its candidate blocks.
+          const unsigned char* bt = Bt + gi * X::B_TILE;
+          auto dist = [&](int k) {           // sum_j (x_j - C_kj)^2 in fp64; the tile holds -2 C in bf16
+            double d2 = 0.0;
+#pragma unroll
+            for (int j8 = 0; j8 < G / 8; ++j8) {
+              const uint4 w = *reinterpret_cast<const uint4*>(bt + kmaj_off(k, j8 * 8, SBO));
+              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float c2 = (e & 1) ? bf16_hi(ww[e >> 1]) : bf16_lo(ww[e >> 1]);
+                const double df = (double)__bfloat162float(xv[j8 * 8 + e]) + 0.5 * (double)c2;
+                d2 = fma(df, df, d2);
+              }
+            }
+            return d2;
+          };
           double best = 1e300;
-          int bk = 0;
-#pragma unroll 1
-          for (int q = 0; q < kEntries / 32; ++q) {
+          int bk = kEntries;
+          if (tie && n_cand <= 3) {
+#pragma unroll
+            for (int c3 = 0; c3 < 3; ++c3) {
+              const int k = (int)((cand >> (9 * c3)) & 511u) - 1;
+              if (k >= 0) {
+                const double d2 = dist(k);
+                if (d2 < best || (d2 == best && k < bk)) { best = d2; bk = k; }
+              }
+            }
+          }
+          const bool many = tie && n_cand > 3;
+          for (uint32_t wm = __reduce_or_sync(0xffffffffu, many ? bmask : 0u); wm; wm &= wm - 1u) {
+            const int q = __ffs(wm) - 1;
             float v[32];
             tmem_ld32(tmem_set + lane_addr + q * 32, v);
-            if (tie) {
-              for (int i = 0; i < 32; ++i) {
+            if (many && ((bmask >> q) & 1u)) {
+#pragma unroll 1
+              for (int i = 0; i < 32; ++i)
                 if (v[i] <= thr) {
                   const int k = q * 32 + i;
-                  const unsigned char* bt = Bt + gi * X::B_TILE;
-                  double d2 = 0.0;
-                  for (int j = 0; j < G; ++j) {
-                    const double cj =
-                        -0.5 * (double)__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(bt + kmaj_off(k, j, SBO)));
-                    const double df = (double)__bfloat162float(xv[j]) - cj;
-                    d2 = fma(df, df, d2);
-                  }
-                  if (d2 < best) { best = d2; bk = k; }
+                  const double d2 = dist(k);
+                  if (d2 < best || (d2 == best && k < bk)) { best = d2; bk = k; }
                 }
-              }
             }
           }
           if (tie) code = bk;
