@@ -63,8 +63,8 @@ def parse():
 # DRAM bytes (read + write) of one decode_kernel<128,4> launch of this workload, from one ncu
 # capture (`python bench.py --profile decode` under ncu), valid only for the decode source it was
 # taken on: the bench reports it when the file's hash still matches, else null.
-DECODE_TRAFFIC = {"source_sha256": "7fb4269e752830ea83cd013c7ecd68a7fcdf147e1eb3db1025a18720edc55ed0",
-                  "bytes_per_launch": 36761088}
+DECODE_TRAFFIC = {"source_sha256": "20698507e7fe49a3228f44041d17f6d36fbc37e270fbcfbb19f9abe1399fb44a",
+                  "bytes_per_launch": 36767744}
 
 
 def decode_traffic():
@@ -81,6 +81,15 @@ def peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def bf16_peak():
+    """Dense bf16 TFLOP/s for a kernel timed on its own (burst figure)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
 
 
 # ------------------------------------------------------------------------------ oracle baseline
@@ -429,7 +438,12 @@ def gpu_arm(args):
         torch.cuda.synchronize()
         enc_ms = a.elapsed_time(b_) / 3
         vectors = wc.ctx * wc.n_kv_heads * 2 * (wc.head_dim // (wc.G // wc.Tc)) * (wc.T // wc.Tc)
+        # useful distance GEMM work: 256 entries x G dims x 2 flops per vector
+        tflops = vectors * 256 * wc.G * 2 / (enc_ms / 1e3) / 1e12
+        tpk, tpk_kind = bf16_peak()
         enc = {"vectors_per_s": vectors / (enc_ms / 1e3), "ms_per_layer": enc_ms,
+               "distance_gemm_tflops": tflops, "frac_of_bf16_peak": tflops / tpk, "bf16_peak": tpk,
+               "peak_kind": tpk_kind,
                "workload": "ouro26_prefill_32k (one of 48 layers)", "kernel": "encode_tc (tcgen05 distance GEMM + argmin)"}
         del kv4, c4
 
