@@ -803,12 +803,25 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
   }
   float* pl2 = SC;              // [np] partial LSEs (log2)
   float* pw = SC + 512;         // [np] partial weights
-  const float lse_i = pl > 0.f ? pm + log2f(pl) : -INFINITY;
-  if (tid < np) pl2[tid] = lse_i;
-  const float M = block_reduce<true>(lse_i, red);
-  const float den = block_reduce<false>(M != -INFINITY && lse_i != -INFINITY ? exp2f(lse_i - M) : 0.f, red);
-  const float Ltot = M == -INFINITY ? -INFINITY : M + log2f(den);
-  if (tid < np) pw[tid] = lse_i == -INFINITY ? 0.f : exp2f(pm - Ltot);
+  if (tid < np) {
+    pl2[tid] = pl > 0.f ? pm + log2f(pl) : -INFINITY;
+    pw[tid] = pm;                                    // replaced by the weight below
+  }
+  __syncthreads();
+  // warp 0: the LSE over the partials and every partial's weight 2^(m_i - L)
+  float Ltot = -INFINITY;
+  if (warp == 0) {
+    float M = -INFINITY;
+    for (int i = lane; i < np; i += 32) M = fmaxf(M, pl2[i]);
+    M = warp_max(M);
+    float den = 0.f;
+    if (M != -INFINITY)
+      for (int i = lane; i < np; i += 32)
+        if (pl2[i] != -INFINITY) den += exp2f(pl2[i] - M);
+    den = warp_sum(den);
+    Ltot = M == -INFINITY ? -INFINITY : M + log2f(den);
+    for (int i = lane; i < np; i += 32) pw[i] = pl2[i] == -INFINITY ? 0.f : exp2f(pw[i] - Ltot);
+  }
   __syncthreads();
   {
     float acc = 0.f;
@@ -829,18 +842,25 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
     }
   }
   constexpr float kLn2 = 0.6931471805599453f;
-  if (tid == 0) {
-    lse[(size_t)b * g.Hq + hq] = Ltot * kLn2;
-    counters[(size_t)b * g.Hq + hq] = 0;
-  }
-  if (split_lse) {
-    float* sl = split_lse + ((size_t)b * g.Hq + hq) * (ns + 1);
-    for (int i = tid; i < ns; i += kThr) sl[i] = pl2[2 * i] * kLn2;
-    // the bf16 partial is the logsumexp of the CTAs' shares
-    const float bl = tid < ns ? pl2[2 * tid + 1] : -INFINITY;
-    const float Bm = block_reduce<true>(bl, red);
-    const float Bs = block_reduce<false>(Bm != -INFINITY && bl != -INFINITY ? exp2f(bl - Bm) : 0.f, red);
-    if (tid == 0) sl[ns] = Bm == -INFINITY ? -INFINITY : (Bm + log2f(Bs)) * kLn2;
+  if (warp == 0) {
+    if (lane == 0) {
+      lse[(size_t)b * g.Hq + hq] = Ltot * kLn2;
+      counters[(size_t)b * g.Hq + hq] = 0;
+    }
+    if (split_lse) {
+      float* sl = split_lse + ((size_t)b * g.Hq + hq) * (ns + 1);
+      for (int i = lane; i < ns; i += 32) sl[i] = pl2[2 * i] * kLn2;
+      // the bf16 partial is the logsumexp of the CTAs' shares
+      float Bm = -INFINITY;
+      for (int i = lane; i < ns; i += 32) Bm = fmaxf(Bm, pl2[2 * i + 1]);
+      Bm = warp_max(Bm);
+      float Bs = 0.f;
+      if (Bm != -INFINITY)
+        for (int i = lane; i < ns; i += 32)
+          if (pl2[2 * i + 1] != -INFINITY) Bs += exp2f(pl2[2 * i + 1] - Bm);
+      Bs = warp_sum(Bs);
+      if (lane == 0) sl[ns] = Bm == -INFINITY ? -INFINITY : (Bm + log2f(Bs)) * kLn2;
+    }
   }
 }
 
