@@ -174,9 +174,9 @@ struct Lane {
 };
 
 template <int D, int C>
-__device__ inline void lane_init(Lane<D, C>& L, int lane, const float* rope, int RC) {
+__device__ inline void lane_init(Lane<D, C>& L, int lane, const float2* etq_s) {
   using X = Dec<D, C>;
-  constexpr int NP = X::NP, TQ = X::TQ, F = X::F;
+  constexpr int NP = X::NP, TQ = X::TQ;
   L.P = lane % NP;
   L.tq = lane / NP;
   L.gb_lo = (uint32_t)L.P * C * 2;
@@ -185,10 +185,9 @@ __device__ inline void lane_init(Lane<D, C>& L, int lane, const float* rope, int
   L.sel[1] = row_sel(L.tq + (TQ == 2 ? 2 : 0));
 #pragma unroll
   for (int e = 0; e < C; ++e) {
-    const int f = L.P * C + e;
-    const float2 r = rope_at(rope, RC, F, TQ, f);
-    L.twoc[e] = make_float2(2.f * r.x, 2.f * r.x);
-    L.mtwoc[e] = make_float2(-2.f * r.x, -2.f * r.x);
+    const float cs = etq_s[L.P * C + e].x;          // cos(TQ theta_f)
+    L.twoc[e] = make_float2(2.f * cs, 2.f * cs);
+    L.mtwoc[e] = make_float2(-2.f * cs, -2.f * cs);
   }
 }
 
@@ -551,6 +550,14 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
   const int nbj = nb > j ? (nb - j + ns - 1) / ns : 0;    // this CTA's share: j, j + ns, ...
   if (producer && lane == 0 && do_coded)
     for (int ci = 0; ci < min(kStages, n_stream); ++ci) issue_chunk(ci);
+  // a compute lane's RoPE factors at its first coded token, fetched now so that their latency
+  // overlaps the prologue
+  float2 rf[C];
+  if (!producer && do_coded) {
+    const int p_first = g.S + n0 + kPage * kPPW * warp + lane / X::NP;
+#pragma unroll
+    for (int e = 0; e < C; ++e) rf[e] = rope_at(rope, g.RC, F, p_first, (lane % X::NP) * C + e);
+  }
   if (!bad && tid < F) {
     const __nv_bfloat16* qv = q + ((size_t)b * g.Hq + hq) * D;
     const float2 qraw = make_float2(__bfloat162float(qv[tid]), __bfloat162float(qv[tid + F]));
@@ -602,14 +609,10 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
     } else {
       // ---- compute warps
       Lane<D, C> L;
-      lane_init<D, C>(L, lane, rope, g.RC);
+      lane_init<D, C>(L, lane, etq_s);
       float2 U[C];                       // W of the lane's first token of the current chunk
-      const int p_first = g.S + n0 + kPage * kPPW * warp + L.tq;
 #pragma unroll
-      for (int e = 0; e < C; ++e) {
-        const int f = L.P * C + e;
-        U[e] = cmul(zq[f], cconj(rope_at(rope, g.RC, F, p_first, f)));
-      }
+      for (int e = 0; e < C; ++e) U[e] = cmul(zq[L.P * C + e], cconj(rf[e]));
       const int pi_own = L.P / X::TPL, t_own = L.tq + TQ * (L.P % X::TPL);   // the lane's token of a run
       const int gv = lane % NG, tp = lane / NG;
       const uint32_t hl = smem_addr(Hs) + (uint32_t)gv * 4;
