@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="lvq", choices=["lvq", "reference"])
     ap.add_argument("--splits", type=int, default=0, help="split count (0: choose)")
+    ap.add_argument("--workload", default=WORKLOAD, choices=["ouro14_g16_32k", "ouro14_g32_b32", "ouro14_tc2_64k"],
+                    help="decode workload (the headline line uses the default)")
     ap.add_argument("--no-encode", action="store_true", help="skip the prefill-encode measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--profile", default="", choices=["", "decode", "encode"],
@@ -199,29 +201,33 @@ class Clocks:
 
 
 def build_cache(w, lvq, synth, torch, extra_tokens: int, device, request_seed: int):
-    """Coded cache at w.ctx context, codes from the library's encoder."""
+    """Coded cache at the workload's per-request contexts, codes from the library's encoder."""
+    ctx = synth.ctx_lengths(w)
+    B = len(ctx)
     cfg = lvq.make_config(w.n_layers, w.n_kv_heads, w.n_q_heads, w.head_dim, w.T, w.Tc, w.G, w.n_sink,
-                          w.n_recent, w.batch, w.ctx + extra_tokens, max_splits=128, rope_base=w.rope_base)
+                          w.n_recent, B, max(ctx) + extra_tokens, max_splits=128, rope_base=w.rope_base)
     cache = lvq.CodedCache(cfg, device)
     lay = cache.lay
-    L = w.ctx - w.n_sink - w.n_recent
+    coded = [c - w.n_sink - w.n_recent for c in ctx]
     cbv, sv, rv = cache.cb_view(), cache.sink_view(), cache.ring_view()
     for layer in range(w.n_layers):
         sc = synth.channel_scales(w, layer, device=device)
         cbv[layer] = synth.codebooks(w, layer, device=device, scales=sc)
-        sk = synth.loop_kv(w, layer, w.n_sink, stream="sink", request=request_seed, device=device, scales=sc)
-        rk = synth.loop_kv(w, layer, lay.ring_tokens, stream="recent", request=request_seed, device=device,
-                           scales=sc)
-        sv[layer, :, :, 0] = sk.permute(0, 1, 3, 2, 4)
-        rv[layer, :, :, 0] = rk.permute(0, 1, 3, 2, 4)
+        for b in range(B):
+            seed = request_seed * B + b
+            sk = synth.loop_kv(w, layer, w.n_sink, stream="sink", request=seed, device=device, scales=sc)
+            rk = synth.loop_kv(w, layer, lay.ring_tokens, stream="recent", request=seed, device=device, scales=sc)
+            sv[layer, :, :, b] = sk.permute(0, 1, 3, 2, 4)
+            rv[layer, :, :, b] = rk.permute(0, 1, 3, 2, 4)
     lvq.lvq_pack_codebooks(cfg, lay, cache.cb, cache.cbp, cache.cb_norm)
     lvq.lvq_rope_table(cfg, lay, cache.rope)
     for layer in range(w.n_layers):
-        kv = synth.loop_kv(w, layer, L, stream="coded", request=request_seed, device=device)
-        lvq.lvq_encode_prefill(cfg, lay, layer, 0, kv, 0, L, 0, cache.cb, cache.idx, cache.status)
-        del kv
-    cache.ctx_len.fill_(w.ctx)
-    cache.coded_len.fill_(L)
+        for b in range(B):
+            kv = synth.loop_kv(w, layer, coded[b], stream="coded", request=request_seed * B + b, device=device)
+            lvq.lvq_encode_prefill(cfg, lay, layer, b, kv, 0, coded[b], 0, cache.cb, cache.idx, cache.status)
+            del kv
+    cache.ctx_len.copy_(torch.tensor(ctx, dtype=torch.int32))
+    cache.coded_len.copy_(torch.tensor(coded, dtype=torch.int32))
     torch.cuda.synchronize()
     cache.check_status("cache build")
     return cfg, cache
@@ -246,17 +252,28 @@ def replica_plan(rank: int, world: int, batch_per_rank: int) -> dict:
 
 
 def choose_splits(w, n_sm: int) -> int:
-    # one CTA per SM: splits * heads * requests <= SMs
-    return max(1, min(128, n_sm // (w.batch * w.n_q_heads)))
+    """Splits per (request, head).  One CTA per SM: when the batch's heads fit in one wave,
+    as many splits as fill it; otherwise splits of about 6K coded tokens, which balance the
+    waves of a ragged batch against each CTA's fixed cost (measured on the 32-request
+    workload: 3-4 splits beat 1, 2 and 6)."""
+    heads = w.batch * w.n_q_heads
+    if heads <= n_sm:
+        return max(1, min(128, n_sm // heads))
+    mean_ctx = w.ctx if w.ctx else (w.ctx_low + w.ctx_high) / 2
+    return max(1, min(16, round(mean_ctx / 6144)))
 
 
-def decode_bytes_per_launch(w, lay, coded: int, recent: int) -> int:
-    """Algorithmic bytes of one decode attention (one layer, one loop step), batch 1."""
-    idx = coded * w.n_kv_heads * 2 * lay.n_groups                 # this step's block rows, K and V
+def decode_bytes_per_launch(w, lay, coded, recent) -> int:
+    """Algorithmic bytes of one decode attention (one layer, one loop step) over the batch:
+    per request its coded rows of this step's block (K and V), its bf16 tokens and its
+    query/output; the step-t codebook slices once per launch."""
     slices = w.n_kv_heads * 2 * 256 * w.head_dim * 2              # step-t codebook slices, K and V
-    bf16 = (min(w.n_sink, coded + recent) + recent) * w.n_kv_heads * 2 * w.head_dim * 2
-    qo = w.n_q_heads * w.head_dim * (2 + 4) + w.n_q_heads * 4
-    return idx + slices + bf16 + qo
+    total = slices
+    for cd, rc in zip(coded, recent):
+        total += cd * w.n_kv_heads * 2 * lay.n_groups             # this step's block rows, K and V
+        total += (min(w.n_sink, cd + rc) + rc) * w.n_kv_heads * 2 * w.head_dim * 2
+        total += w.n_q_heads * w.head_dim * (2 + 4) + w.n_q_heads * 4
+    return total
 
 
 def profile_encode(lvq, synth, torch, device):
@@ -295,7 +312,7 @@ def gpu_arm(args):
     if args.profile == "encode":
         profile_encode(lvq, synth, torch, device)
         return
-    w = synth.WORKLOADS[WORKLOAD]
+    w = synth.WORKLOADS[args.workload]
     replays = 2 * args.steps + args.warmup + 3          # every graph replay adds 8 tokens
     cfg, cache = build_cache(w, lvq, synth, torch, TOKENS_PER_STEP * (replays + 4), device,
                              replica_plan(rank, world, w.batch)["seed"])
@@ -369,8 +386,8 @@ def gpu_arm(args):
     value = tokens / (ms / 1e3)
 
     # ---- decode kernel timing: a graph of the 96 attentions of one token, event-timed
-    coded_now = int(cache.coded_len[0].item())
-    ctx_now = int(cache.ctx_len[0].item())
+    coded_now = [int(v) for v in cache.coded_len[:B].tolist()]
+    ctx_now = [int(v) for v in cache.ctx_len[:B].tolist()]
     g2 = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g2, stream=stream):
         for t in range(w.T):
@@ -390,11 +407,11 @@ def gpu_arm(args):
         e1.record(stream)
     torch.cuda.synchronize()
     per_call_ms = e0.elapsed_time(e1) / (reps * NL)
-    recent_now = ctx_now - w.n_sink - coded_now
+    recent_now = [c - w.n_sink - cd for c, cd in zip(ctx_now, coded_now)]
     bpl = decode_bytes_per_launch(w, lay, coded_now, recent_now)
     hbm_peak, peak_kind = peaks()
     achieved = bpl / (per_call_ms / 1e3) / 1e9
-    code_stream = coded_now * w.n_kv_heads * 2 * lay.n_groups / (per_call_ms / 1e3) / 1e9
+    code_stream = sum(coded_now) * w.n_kv_heads * 2 * lay.n_groups / (per_call_ms / 1e3) / 1e9
 
     # ---- e2e: queries in from pinned host memory, outputs back, every step
     q_host = torch.empty(q_all.shape, dtype=q_all.dtype).pin_memory()
@@ -457,12 +474,16 @@ def gpu_arm(args):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "global_batch": B * world, "seq_len": w.ctx, "layers": w.n_layers,
+        "config": {"workload": args.workload, "global_batch": B * world,
+                   "seq_len": w.ctx if w.ctx else f"{w.ctx_low}-{w.ctx_high}", "layers": w.n_layers,
                    "loop_steps": w.T, "Tc": w.Tc, "G": w.G, "kv_heads": w.n_kv_heads, "head_dim": d,
                    "num_splits": ns, "tokens_per_step": TOKENS_PER_STEP,
-                   "l2": "inputs larger than L2 (3.5 GB of codes per token)", "parallelism": f"replicas{world}"},
+                   "l2": f"inputs larger than L2 ({NL * bpl / 1e9:.1f} GB read per generated token)",
+                   "parallelism": f"replicas{world}"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": decode_traffic(), "kernel": "decode_kernel<128,4>",
+                     "frac": achieved / hbm_peak,
+                     "traffic": decode_traffic() if args.workload == WORKLOAD else None,
+                     "kernel": f"decode_kernel<{d},{lay.c}>",
                      "peak_kind": peak_kind, "bytes_per_launch": bpl, "launch_ms": per_call_ms},
         "code_stream_GBps": code_stream,
         "cpu_baseline": cb,
