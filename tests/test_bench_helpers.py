@@ -1,0 +1,39 @@
+"""Host-side helpers of bench.py: the split choice and the algorithmic byte model that the
+roofline line divides by (closed forms of the cache layout)."""
+import dataclasses
+
+import bench
+from sub_bit_kv_b200 import synth
+
+
+class _Lay:
+    def __init__(self, n_groups):
+        self.n_groups = n_groups
+
+
+def test_decode_bytes_closed_form_32k():
+    w = synth.WORKLOADS["ouro14_g16_32k"]
+    coded, recent = 32636, 128
+    got = bench.decode_bytes_per_launch(w, _Lay(32), [coded], [recent])
+    idx = coded * 16 * 2 * 32                 # 32 code bytes per token, head and K/V
+    slices = 16 * 2 * 256 * 128 * 2           # step-t K/V slices of the 16 heads
+    bf16 = (4 + 128) * 16 * 2 * 128 * 2       # sink + recent tokens, K and V
+    qo = 16 * 128 * (2 + 4) + 16 * 4          # bf16 query in, fp32 output and lse out
+    assert got == idx + slices + bf16 + qo == 36_610_112
+
+
+def test_decode_bytes_batch_counts_slices_once():
+    w = synth.WORKLOADS["ouro14_g32_b32"]
+    one = bench.decode_bytes_per_launch(w, _Lay(16), [1000], [128])
+    two = bench.decode_bytes_per_launch(w, _Lay(16), [1000, 1000], [128, 128])
+    slices = 16 * 2 * 256 * 128 * 2
+    assert two - one == one - slices
+
+
+def test_choose_splits():
+    ws = synth.WORKLOADS
+    assert bench.choose_splits(ws["ouro14_g16_32k"], 148) == 9         # 16 heads fill one wave
+    assert bench.choose_splits(ws["ouro14_tc2_64k"], 148) == 1         # 128 heads already fill it
+    assert bench.choose_splits(ws["ouro14_g32_b32"], 148) == 3         # 512 heads: ~6K-token splits
+    tiny = dataclasses.replace(ws["tiny"], batch=1)
+    assert bench.choose_splits(tiny, 148) == 128                        # capped
