@@ -42,6 +42,9 @@ constexpr int kTileTokens = 128;
 constexpr int kItemTokens = 1024;   // tokens per work item (8 tiles)
 constexpr int kSpan = 16;           // channels per item (TMA box x: 32 bytes)
 constexpr int kRawStages = 2;
+// a thread's copy of one 32-column block: 32 floats + 4 of padding, so that eight
+// consecutive threads' 16-byte accesses fall in distinct bank groups
+constexpr int kKeepStride = 36;
 
 template <int G, int C>
 struct Enc {
@@ -59,7 +62,8 @@ struct Enc {
   static constexpr int OFF_NMAX = OFF_RAW + kRawStages * RAW;
   static constexpr int OFF_BAR = OFF_NMAX + 16 * 4;
   static constexpr int OFF_BMIN = OFF_BAR + 8 * (kRawStages + 2);     // [8][256] block minima
-  static constexpr int OFF_TMEM = OFF_BMIN + (kEntries / 32) * kThreads * 4;
+  static constexpr int OFF_KEEP = OFF_BMIN + (kEntries / 32) * kThreads * 4;   // [256][kKeepStride]
+  static constexpr int OFF_TMEM = OFF_KEEP + kThreads * kKeepStride * 4;
   // + alignment slack; at least 120 KB so that one CTA (holding all of TMEM) fits per SM
   static constexpr int SMEM = (OFF_TMEM + 16 + 1024) > 120 * 1024 ? (OFF_TMEM + 16 + 1024) : 120 * 1024;
   static_assert(NGC == 2 || NGC == 4, "two MMA sets alternate over the item's groups");
@@ -166,6 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + X::OFF_TMEM);
   volatile int* fail_s = reinterpret_cast<volatile int*>(smem + X::OFF_TMEM + 4);   // per MMA set
   float* bmin_s = reinterpret_cast<float*>(smem + X::OFF_BMIN);
+  float* keep_s = reinterpret_cast<float*>(smem + X::OFF_KEEP);
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int set = tid / kRows;            // MMA set: warps 0-3 or 4-7
@@ -311,10 +316,14 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
         named_sync(1 + set, kRows);
         const bool ok = fail_s[set] == 0;      // uniform over the set
 
-        // epilogue: the row's minimum with the minimum of every 32-column block (one wait per 64
-        // columns), then the candidates within eps of it -- only blocks whose minimum is within
-        // eps can hold one, so usually a single block is read again
+        // epilogue, one pass over TMEM: the minimum of every 32-column block, and the
+        // block holding the running minimum copied to this thread's slot in shared
+        // memory; then the candidates (within eps of the row minimum) are counted from the
+        // block minima and, inside the kept block, from the copy -- no second TMEM pass
         const float eps = ldexpf(xx + nmax_s[gi], -14);
+        float* keep = keep_s + tid * kKeepStride;
+        float run = __int_as_float(0x7f800000);   // +inf
+        int run_b = 0;
 #pragma unroll 1
         for (int q2 = 0; q2 < kEntries / 64; ++q2) {
           uint32_t ra[64];
@@ -330,46 +339,34 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
               m1 = fmin3(m1, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
             }
             m0 = fmin3(m0, __uint_as_float(r[30]), __uint_as_float(r[31]));
-            bmin_s[(2 * q2 + b2) * kThreads + tid] = fminf(m0, m1);
+            const float bm = fminf(m0, m1);
+            bmin_s[(2 * q2 + b2) * kThreads + tid] = bm;
+            if (bm < run) {                            // strict: the first block of equal minima
+              run = bm;
+              run_b = 2 * q2 + b2;
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<uint4*>(keep + 4 * j) = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+            }
           }
         }
-        float bmin[kEntries / 32];
-#pragma unroll
-        for (int q = 0; q < kEntries / 32; ++q) bmin[q] = bmin_s[q * kThreads + tid];
-        float mrow = bmin[0];
-#pragma unroll
-        for (int q = 1; q < kEntries / 32; ++q) mrow = fminf(mrow, bmin[q]);
-        const float thr = mrow + eps;
+        const float thr = run + eps;
         uint32_t bmask = 0;                // blocks that can hold a candidate of this row
 #pragma unroll
-        for (int q = 0; q < kEntries / 32; ++q) bmask |= (bmin[q] <= thr ? 1u : 0u) << q;
-        uint32_t cand = 0;                 // (k+1) of the last 3 candidates, 9 bits each, last in the low bits
-        int n_cand = 0;
-        // the 64-column pairs of blocks any row of the warp needs, in order (tcgen05.ld is
-        // warp-collective); one wait per pair
-        uint32_t pairs = __reduce_or_sync(0xffffffffu, bmask);
-        pairs = (pairs | (pairs >> 1)) & 0x55u;
-        for (; pairs; pairs &= pairs - 1u) {
-          const int q = __ffs(pairs) - 1;           // even: blocks q and q + 1
-          uint32_t r[64];
-          tmem_ld64_nowait(tmem_set + lane_addr + q * 32, r);
-          tmem_wait_ld();
+        for (int q = 0; q < kEntries / 32; ++q) bmask |= (bmin_s[q * kThreads + tid] <= thr ? 1u : 0u) << q;
+        uint32_t m = 0u;                   // candidates inside the kept block
 #pragma unroll
-          for (int b2 = 0; b2 < 2; ++b2)
-            if ((bmask >> (q + b2)) & 1u) {
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (__uint_as_float(r[32 * b2 + i]) <= thr) {
-                  cand = (cand << 9) + (uint32_t)((q + b2) * 32 + i + 1);
-                  ++n_cand;
-                }
-            }
+        for (int j = 0; j < 8; ++j) {
+          const float4 v = *reinterpret_cast<const float4*>(keep + 4 * j);
+          m |= ((v.x <= thr ? 1u : 0u) | (v.y <= thr ? 2u : 0u) | (v.z <= thr ? 4u : 0u) | (v.w <= thr ? 8u : 0u))
+               << (4 * j);
         }
-        int code = (int)(cand & 511u) - 1;
+        int code = run_b * 32 + __ffs(m) - 1;
+        const int n_cand = __popc(m) + __popc(bmask & ~(1u << run_b));
         const bool tie = n_cand > 1;
         if (__any_sync(0xffffffffu, tie && valid_row)) {
-          // near-tie: exact fp64 direct-form distances of the candidates, lowest index on ties.
-          // Up to 3 candidates are in `cand`; a row with more rescans its candidate blocks.
+          // near-tie: exact fp64 direct-form distances of the candidates (the row's candidate
+          // blocks are read again), lowest index on ties
           const unsigned char* bt = Bt + gi * X::B_TILE;
           auto dist = [&](int k) {           // sum_j (x_j - C_kj)^2 in fp64; the tile holds -2 C in bf16
             double d2 = 0.0;
@@ -388,29 +385,18 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
           };
           double best = 1e300;
           int bk = kEntries;
-          if (tie && n_cand <= 3) {
-#pragma unroll
-            for (int c3 = 0; c3 < 3; ++c3) {
-              const int k = (int)((cand >> (9 * c3)) & 511u) - 1;
-              if (k >= 0) {
-                const double d2 = dist(k);
-                if (d2 < best || (d2 == best && k < bk)) { best = d2; bk = k; }
-              }
-            }
-          }
-          const bool many = tie && n_cand > 3;
-          for (uint32_t wm = __reduce_or_sync(0xffffffffu, many ? bmask : 0u); wm; wm &= wm - 1u) {
+          for (uint32_t wm = __reduce_or_sync(0xffffffffu, tie ? bmask : 0u); wm; wm &= wm - 1u) {
             const int q = __ffs(wm) - 1;
             float v[32];
             tmem_ld32(tmem_set + lane_addr + q * 32, v);
-            if (many && ((bmask >> q) & 1u)) {
-#pragma unroll 1
-              for (int i = 0; i < 32; ++i)
-                if (v[i] <= thr) {
-                  const int k = q * 32 + i;
-                  const double d2 = dist(k);
-                  if (d2 < best || (d2 == best && k < bk)) { best = d2; bk = k; }
-                }
+            uint32_t m = 0u;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) m |= (v[i] <= thr ? 1u : 0u) << i;
+            if (!tie || !((bmask >> q) & 1u)) m = 0u;
+            for (; m; m &= m - 1u) {
+              const int k = q * 32 + __ffs(m) - 1;
+              const double d2 = dist(k);
+              if (d2 < best || (d2 == best && k < bk)) { best = d2; bk = k; }
             }
           }
           if (tie) code = bk;

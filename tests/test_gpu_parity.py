@@ -74,6 +74,44 @@ def test_encode_prefill_matches_oracle(name, ntok, offset, extra):
     print(f"{name}: near-ties {ties}")
 
 
+@pytest.mark.parametrize("name,extra", [
+    ("ouro14_g16_32k", {"n_kv_heads": 2, "n_q_heads": 2}),     # G = 16, c = 4 (tensor-core encoder)
+    ("ouro14_g32_b32", {"n_kv_heads": 2, "n_q_heads": 2}),     # G = 32, c = 8
+])
+def test_encode_prefill_duplicate_entries_lowest_index(name, extra):
+    """Exact ties: entries 128..191 repeat entries 0..63 (the twin lies four 32-entry blocks
+    later) and entry 64+2j+1 repeats entry 64+2j (twins inside one block).  The direct form
+    ranks twins equal, so the code is the lower index of the pair wherever a twin is nearest
+    (the nearest-entry rule of the method, lowest index on ties)."""
+    w = _reduced(name, n_layers=1, **extra)
+    ntok = 700
+    case = Hl.build_case(w, layers=1, ctx=[w.n_sink + ntok + w.n_recent], coded=[ntok], codes_from="none")
+    c = case.cache
+    cb = case.cb[0].clone()                                  # [2][n_blk][H][n_g][256][G]
+    cb[..., 128:192, :] = cb[..., 0:64, :]
+    cb[..., 65:128:2, :] = cb[..., 64:128:2, :]
+    c.cb_view()[0] = cb.cuda()
+    kv = synth.loop_kv(w, 0, ntok, stream="enc")
+    lvq.lvq_encode_prefill(case.cfg, c.lay, 0, 0, kv.cuda(), 0, ntok, 0, c.cb, c.idx, c.status)
+    torch.cuda.synchronize()
+    c.check_status()
+    cbf = Hl.f64(cb)
+    x = Hl.f64(kv)
+    exact_ties = 0
+    for kvi in range(2):
+        got = Hl.get_codes(c, 0, 0, kvi, 0, ntok).numpy()    # [n_blk][N][H][n_g]
+        X = O.joint_vectors(x[kvi], w.Tc, w.G)
+        for blk in range(X.shape[0]):
+            for h in range(X.shape[2]):
+                for g in range(X.shape[3]):
+                    ref, d1, d2 = O.nearest_entry(X[blk, :, h, g], cbf[kvi, blk, h, g])
+                    twin = d2 == d1
+                    assert (got[blk, twin, h, g] == ref[twin]).all()
+                    exact_ties += int(twin.sum())
+                    check_codes(got[blk, :, h, g], X[blk, :, h, g], cbf[kvi, blk, h, g])
+    assert exact_ties > 0
+
+
 def test_codebook_entries_reencode_to_own_index():
     w = synth.WORKLOADS["tiny"]
     case = Hl.build_case(w, layers=1, ctx=[w.n_sink + 256 + w.n_recent], coded=[256], codes_from="none")
