@@ -20,13 +20,14 @@
 // direct form sum_j (X_j - C_kj)^2 -- exact for bf16 inputs -- lowest index on
 // ties.  So every code equals the fp64 brute-force answer.
 //
-// CTA: 256 threads, one per SM (it allocates all 512 TMEM columns).  Work items
+// CTA: 512 threads, one per SM (it allocates all 512 TMEM columns).  Work items
 // are (K/V, block, head, 16-channel span) x 1024-token ranges.  The raw input
 // tile [Tc][128 tokens][16 channels] arrives by TMA (no multicast) into a
-// 2-stage ring; the 16 channels hold 16/c groups.  Two sets of 4 warps (one
-// per TMEM lane quadrant) each own 256 TMEM columns and alternate over the
-// groups: build the group's A tile, issue its UMMA, and run the argmin
-// epilogue, so one set's epilogue overlaps the other set's MMA.
+// 2-stage ring; the 16 channels hold 16/c groups.  Two sets of 8 warps each own
+// 256 TMEM columns and alternate over the groups: build the group's A tile,
+// issue its UMMA, and run the argmin epilogue, so one set's epilogue overlaps
+// the other set's MMA.  In a set, warps w and w + 4 read the same TMEM lane
+// quadrant (32 rows) and split the 256 entries into halves.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -36,15 +37,13 @@ namespace lvq {
 
 namespace tc {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
+constexpr int kSetThreads = 256;    // one MMA set: 8 warps
 constexpr int kRows = 128;          // UMMA M
 constexpr int kTileTokens = 128;
 constexpr int kItemTokens = 1024;   // tokens per work item (8 tiles)
 constexpr int kSpan = 16;           // channels per item (TMA box x: 32 bytes)
 constexpr int kRawStages = 2;
-// a thread's copy of one 32-column block: 32 floats + 4 of padding, so that eight
-// consecutive threads' 16-byte accesses fall in distinct bank groups
-constexpr int kKeepStride = 36;
 
 template <int G, int C>
 struct Enc {
@@ -61,12 +60,13 @@ struct Enc {
   static constexpr int OFF_RAW = OFF_A + NGC * A_TILE;
   static constexpr int OFF_NMAX = OFF_RAW + kRawStages * RAW;
   static constexpr int OFF_BAR = OFF_NMAX + 16 * 4;
-  static constexpr int OFF_BMIN = OFF_BAR + 8 * (kRawStages + 2);     // [8][256] block minima
-  static constexpr int OFF_KEEP = OFF_BMIN + (kEntries / 32) * kThreads * 4;   // [256][kKeepStride]
-  static constexpr int OFF_TMEM = OFF_KEEP + kThreads * kKeepStride * 4;
+  static constexpr int OFF_BMIN = OFF_BAR + 8 * (kRawStages + 2);     // [2 sets][8 blocks][128 rows]
+  static constexpr int OFF_MASK = OFF_BMIN + 2 * (kEntries / 32) * kRows * 4;   // [2 sets][2 halves][128 rows]
+  static constexpr int OFF_TMEM = OFF_MASK + 2 * 2 * kRows * 4;
   // + alignment slack; at least 120 KB so that one CTA (holding all of TMEM) fits per SM
   static constexpr int SMEM = (OFF_TMEM + 16 + 1024) > 120 * 1024 ? (OFF_TMEM + 16 + 1024) : 120 * 1024;
   static_assert(NGC == 2 || NGC == 4, "two MMA sets alternate over the item's groups");
+  static_assert(SMEM <= 227 * 1024, "shared memory of one CTA");
   static_assert(KP % 16 == 0, "K steps");
 };
 
@@ -91,6 +91,14 @@ __device__ inline void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, 
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
       :: "r"(dst), "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar) : "memory");
+}
+
+// byte offset of channel ch of token row r (of step s) in a raw tile written by TMA with
+// the 32-byte swizzle: each token row is 32 bytes, and its two 16-byte halves trade
+// places when bit 2 of r is set (address bit 4 ^= bit 7), so that eight consecutive
+// rows' 16-byte halves fall in distinct bank groups
+__device__ inline uint32_t raw_off(int s, int r, int ch) {
+  return (uint32_t)((s * kTileTokens + r) * 32 + ((((ch >> 3) ^ (r >> 2)) & 1) << 4) + (ch & 7) * 2);
 }
 
 __device__ inline void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
@@ -157,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
     const __grid_constant__ CUtensorMap tmap, Geo g, int layer, int req, int tok_begin, int n_tok,
     int coded_offset, const __nv_bfloat16* __restrict__ cb, uint8_t* __restrict__ idx, int32_t* st) {
   using X = Enc<G, C>;
-  constexpr int TC = X::TC, NGC = X::NGC, KP = X::KP, SBO = X::SBO;
+  constexpr int TC = X::TC, NGC = X::NGC, SBO = X::SBO;
   extern __shared__ unsigned char smem_raw[];
   // 1024-byte alignment of the dynamic shared memory base
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -170,11 +178,13 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + X::OFF_TMEM);
   volatile int* fail_s = reinterpret_cast<volatile int*>(smem + X::OFF_TMEM + 4);   // per MMA set
   float* bmin_s = reinterpret_cast<float*>(smem + X::OFF_BMIN);
-  float* keep_s = reinterpret_cast<float*>(smem + X::OFF_KEEP);
+  uint32_t* mask_s = reinterpret_cast<uint32_t*>(smem + X::OFF_MASK);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int set = tid / kRows;            // MMA set: warps 0-3 or 4-7
-  const int row = tid % kRows;            // TMEM lane = tile row = token of the tile
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int set = tid / kSetThreads;      // MMA set: warps 0-7 or 8-15
+  const int hf = (warp >> 2) & 1;         // half of the 256 entries this warp scans
+  const int row = 32 * (warp & 3) + lane; // TMEM lane = tile row = token of the tile
+  const bool set_leader = (tid % kSetThreads) == 0;
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" :: "r"(smem_addr(tmem_slot))
@@ -196,6 +206,8 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t tmem_set = tmem_base + (uint32_t)(set * 256);
   const uint32_t lane_addr = ((uint32_t)(32 * (warp & 3))) << 16;
+  float* const bmin_set = bmin_s + set * (kEntries / 32) * kRows;     // [8 blocks][128 rows]
+  uint32_t* const mask_set = mask_s + set * 2 * kRows;                // [2 halves][128 rows]
 
   const int n_spans = g.d / kSpan;
   const int n_sets = 2 * g.nblk * g.H * n_spans;
@@ -237,24 +249,32 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
     for (int e = tid; e < NGC * kEntries; e += kThreads) {
       const int gi = e / kEntries, k = e % kEntries;
       const int grp = span * NGC + gi;
-      const __nv_bfloat16* ce = cb + cb_off(g, layer, kvi, blk, h, grp) + (size_t)k * G;
+      const uint4* ce = reinterpret_cast<const uint4*>(cb + cb_off(g, layer, kvi, blk, h, grp) + (size_t)k * G);
       unsigned char* bt = Bt + gi * X::B_TILE;
       double n = 0.0;
 #pragma unroll
-      for (int j = 0; j < G; ++j) {
-        const float v = __bfloat162float(ce[j]);
-        n += (double)v * (double)v;
-        *reinterpret_cast<__nv_bfloat16*>(bt + kmaj_off(k, j, SBO)) = __float2bfloat16_rn(-2.f * v);
+      for (int j8 = 0; j8 < G / 8; ++j8) {
+        const uint4 w = __ldg(ce + j8);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float lo = bf16_lo(ww[q]), hi = bf16_hi(ww[q]);
+          n = fma((double)lo, (double)lo, n);
+          n = fma((double)hi, (double)hi, n);
+          const __nv_bfloat162 m2 = __floats2bfloat162_rn(-2.f * lo, -2.f * hi);   // exact
+          o[q] = *reinterpret_cast<const uint32_t*>(&m2);
+        }
+        *reinterpret_cast<uint4*>(bt + kmaj_off(k, j8 * 8, SBO)) = make_uint4(o[0], o[1], o[2], o[3]);
       }
       const __nv_bfloat16 n1 = __double2bfloat16(n);
       const double r1 = n - (double)__bfloat162float(n1);
       const __nv_bfloat16 n2 = __double2bfloat16(r1);
       const __nv_bfloat16 n3 = __double2bfloat16(r1 - (double)__bfloat162float(n2));
-      *reinterpret_cast<__nv_bfloat16*>(bt + kmaj_off(k, G, SBO)) = n1;
-      *reinterpret_cast<__nv_bfloat16*>(bt + kmaj_off(k, G + 1, SBO)) = n2;
-      *reinterpret_cast<__nv_bfloat16*>(bt + kmaj_off(k, G + 2, SBO)) = n3;
-      for (int j = G + 3; j < KP; ++j)
-        *reinterpret_cast<__nv_bfloat16*>(bt + kmaj_off(k, j, SBO)) = __float2bfloat16_rn(0.f);
+      *reinterpret_cast<uint4*>(bt + kmaj_off(k, G, SBO)) =
+          make_uint4((uint32_t)__bfloat16_as_ushort(n1) | ((uint32_t)__bfloat16_as_ushort(n2) << 16),
+                     (uint32_t)__bfloat16_as_ushort(n3), 0u, 0u);
+      *reinterpret_cast<uint4*>(bt + kmaj_off(k, G + 8, SBO)) = make_uint4(0u, 0u, 0u, 0u);
       atomicMax(reinterpret_cast<int*>(&nmax_s[gi]), __float_as_int((float)n));
     }
     fence_proxy_async();
@@ -273,37 +293,47 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
 
       // each set handles groups gi = set, set + 2, ...
       for (int gi = set; gi < NGC; gi += 2) {
-        // A row: joint vector of token t0+row, group gi: element s*c+e = raw[s][row][gi*c+e]
+        // A row: joint vector of token t0+row, group gi: element s*c+e = raw[s][row][gi*c+e].
+        // Both threads of a row read it (for ||x||^2); each writes half of its 16-byte chunks.
         unsigned char* at = At + gi * X::A_TILE;
         float xx = 0.f;
-        __nv_bfloat16 xv[G];
+        {
+          uint32_t xw[G / 2];                  // the row's G elements, two per word
 #pragma unroll
-        for (int s2 = 0; s2 < TC; ++s2)
-#pragma unroll
-          for (int e = 0; e < C; ++e) {
-            const __nv_bfloat16 v =
-                *reinterpret_cast<const __nv_bfloat16*>(rw + ((s2 * kTileTokens + row) * kSpan + gi * C + e) * 2);
-            xv[s2 * C + e] = v;
-            const float f = __bfloat162float(v);
-            xx = fmaf(f, f, xx);
+          for (int s2 = 0; s2 < TC; ++s2) {
+            const unsigned char* src = rw + raw_off(s2, row, gi * C);
+            if constexpr (C == 4) {
+              const uint2 w = *reinterpret_cast<const uint2*>(src);
+              xw[s2 * 2] = w.x;
+              xw[s2 * 2 + 1] = w.y;
+            } else {
+              const uint4 w = *reinterpret_cast<const uint4*>(src);
+              xw[s2 * 4] = w.x;
+              xw[s2 * 4 + 1] = w.y;
+              xw[s2 * 4 + 2] = w.z;
+              xw[s2 * 4 + 3] = w.w;
+            }
           }
 #pragma unroll
-        for (int k8 = 0; k8 < G / 8; ++k8) {
-          auto pk = [&](int q) {
-            return (uint32_t)__bfloat16_as_ushort(xv[k8 * 8 + 2 * q]) |
-                   ((uint32_t)__bfloat16_as_ushort(xv[k8 * 8 + 2 * q + 1]) << 16);
-          };
-          *reinterpret_cast<uint4*>(at + kmaj_off(row, k8 * 8, SBO)) = make_uint4(pk(0), pk(1), pk(2), pk(3));
-        }
-        {
-          const uint32_t one = 0x3f80u;   // bf16 1.0
-          uint4 w = make_uint4(one | (one << 16), one, 0u, 0u);
-          *reinterpret_cast<uint4*>(at + kmaj_off(row, G, SBO)) = w;
+          for (int q = 0; q < G / 2; ++q) {
+            const float lo = bf16_lo(xw[q]), hi = bf16_hi(xw[q]);
+            xx = fmaf(lo, lo, xx);
+            xx = fmaf(hi, hi, xx);
+          }
+#pragma unroll
+          for (int k8 = 0; k8 < G / 8; ++k8)
+            if ((k8 >= G / 16) == (hf == 1))
+              *reinterpret_cast<uint4*>(at + kmaj_off(row, k8 * 8, SBO)) =
+                  make_uint4(xw[k8 * 4], xw[k8 * 4 + 1], xw[k8 * 4 + 2], xw[k8 * 4 + 3]);
+          if (hf == 1) {
+            const uint32_t one = 0x3f80u;   // bf16 1.0
+            *reinterpret_cast<uint4*>(at + kmaj_off(row, G, SBO)) = make_uint4(one | (one << 16), one, 0u, 0u);
+          }
         }
         fence_proxy_async();
         tc_fence_before();
-        named_sync(1 + set, kRows);
-        if (row == 0) {
+        named_sync(1 + set, kSetThreads);
+        if (set_leader) {
           tc_fence_after();
           const uint32_t a0 = smem_addr(at), b0 = smem_addr(Bt + gi * X::B_TILE);
 #pragma unroll
@@ -311,23 +341,26 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
             mma_bf16(tmem_set, smem_desc(a0 + ks * 256, SBO), smem_desc(b0 + ks * 256, SBO), kIdesc, ks > 0);
           mma_commit(smem_addr(&bars[kRawStages + set]));
         }
-        if (!mbar_wait(smem_addr(&bars[kRawStages + set]), mma_phase, kWaitIters)) fail_s[set] = 1;
+        // one warp of the set waits for the MMA; the barrier releases the others (no spinning)
+        if ((tid % kSetThreads) < 32) {
+          __syncwarp();
+          if (!mbar_wait(smem_addr(&bars[kRawStages + set]), mma_phase, kWaitIters)) fail_s[set] = 1;
+        }
+        named_sync(1 + set, kSetThreads);
         tc_fence_after();
-        named_sync(1 + set, kRows);
-        const bool ok = fail_s[set] == 0;      // uniform over the set
 
-        // epilogue, one pass over TMEM: the minimum of every 32-column block, and the
-        // block holding the running minimum copied to this thread's slot in shared
-        // memory; then the candidates (within eps of the row minimum) are counted from the
-        // block minima and, inside the kept block, from the copy -- no second TMEM pass
+        // epilogue, one pass over this warp's half of the row (four 32-column blocks, two
+        // 64-column loads): each block's minimum, and the block's columns within eps of that
+        // minimum as a bit mask (bit 31 - i for column i).  Of the block holding the row
+        // minimum, that mask is exactly the row's candidates inside it; any other block whose
+        // minimum is within eps of the row minimum holds further candidates.
         const float eps = ldexpf(xx + nmax_s[gi], -14);
-        float* keep = keep_s + tid * kKeepStride;
-        float run = __int_as_float(0x7f800000);   // +inf
-        int run_b = 0;
+        float hbest = __int_as_float(0x7f800000);   // +inf
+        uint32_t hmask = 0u;                        // candidate mask of this half's best block
 #pragma unroll 1
-        for (int q2 = 0; q2 < kEntries / 64; ++q2) {
+        for (int q2 = 0; q2 < 2; ++q2) {
           uint32_t ra[64];
-          tmem_ld64_nowait(tmem_set + lane_addr + q2 * 64, ra);
+          tmem_ld64_nowait(tmem_set + lane_addr + hf * 128 + q2 * 64, ra);
           tmem_wait_ld();
 #pragma unroll
           for (int b2 = 0; b2 < 2; ++b2) {
@@ -340,47 +373,62 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
             }
             m0 = fmin3(m0, __uint_as_float(r[30]), __uint_as_float(r[31]));
             const float bm = fminf(m0, m1);
-            bmin_s[(2 * q2 + b2) * kThreads + tid] = bm;
-            if (bm < run) {                            // strict: the first block of equal minima
-              run = bm;
-              run_b = 2 * q2 + b2;
+            bmin_set[(hf * 4 + q2 * 2 + b2) * kRows + row] = bm;
+            // sign of (bm + eps) - v per column, shifted in: 1 = outside the window
+            const float tb = bm + eps;
+            const float2 t2 = make_float2(tb, tb), neg1 = make_float2(-1.f, -1.f);
+            uint32_t sg = 0u;
 #pragma unroll
-              for (int j = 0; j < 8; ++j)
-                *reinterpret_cast<uint4*>(keep + 4 * j) = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+            for (int i = 0; i < 32; i += 2) {
+              const float2 e = __ffma2_rn(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), neg1, t2);
+              sg = __funnelshift_l(__float_as_uint(e.x), sg, 1);
+              sg = __funnelshift_l(__float_as_uint(e.y), sg, 1);
+            }
+            if (bm < hbest) {                          // strict: the first block of equal minima
+              hbest = bm;
+              hmask = ~sg;
             }
           }
         }
-        const float thr = run + eps;
-        uint32_t bmask = 0;                // blocks that can hold a candidate of this row
+        mask_set[hf * kRows + row] = hmask;
+        named_sync(1 + set, kSetThreads);      // also: every thread saw the MMA wait's outcome
+        const bool ok = fail_s[set] == 0;      // uniform over the set
+        float bmin[kEntries / 32];
 #pragma unroll
-        for (int q = 0; q < kEntries / 32; ++q) bmask |= (bmin_s[q * kThreads + tid] <= thr ? 1u : 0u) << q;
-        uint32_t m = 0u;                   // candidates inside the kept block
+        for (int q = 0; q < kEntries / 32; ++q) bmin[q] = bmin_set[q * kRows + row];
+        float mrow = bmin[0];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float4 v = *reinterpret_cast<const float4*>(keep + 4 * j);
-          m |= ((v.x <= thr ? 1u : 0u) | (v.y <= thr ? 2u : 0u) | (v.z <= thr ? 4u : 0u) | (v.w <= thr ? 8u : 0u))
-               << (4 * j);
+        for (int q = 1; q < kEntries / 32; ++q) mrow = fminf(mrow, bmin[q]);
+        const float thr = mrow + eps;
+        uint32_t bmask = 0, at_min = 0;   // blocks that can hold a candidate / that hold the minimum
+#pragma unroll
+        for (int q = 0; q < kEntries / 32; ++q) {
+          bmask |= (bmin[q] <= thr ? 1u : 0u) << q;
+          at_min |= (bmin[q] == mrow ? 1u : 0u) << q;
         }
-        int code = run_b * 32 + __ffs(m) - 1;
-        const int n_cand = __popc(m) + __popc(bmask & ~(1u << run_b));
-        const bool tie = n_cand > 1;
+        const int wb = at_min ? __ffs(at_min) - 1 : 0;   // the first block holding the minimum
+        const bool mine = (wb >> 2) == hf;     // this thread's half holds it: it owns the row
+        const uint32_t cm = mask_set[(wb >> 2) * kRows + row];
+        int code = wb * 32 + __clz(cm);
+        const bool tie = mine && (__popc(cm) + __popc(bmask & ~(1u << wb)) > 1);
         if (__any_sync(0xffffffffu, tie && valid_row)) {
-          // near-tie: exact fp64 direct-form distances of the candidates (the row's candidate
-          // blocks are read again), lowest index on ties
+          // near-tie: exact fp64 direct-form distances of every candidate (the row's candidate
+          // blocks are read again, from either half), lowest index on ties
           const unsigned char* bt = Bt + gi * X::B_TILE;
           auto dist = [&](int k) {           // sum_j (x_j - C_kj)^2 in fp64; the tile holds -2 C in bf16
             double d2 = 0.0;
 #pragma unroll
-            for (int j8 = 0; j8 < G / 8; ++j8) {
-              const uint4 w = *reinterpret_cast<const uint4*>(bt + kmaj_off(k, j8 * 8, SBO));
-              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+            for (int s2 = 0; s2 < TC; ++s2)
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const float c2 = (e & 1) ? bf16_hi(ww[e >> 1]) : bf16_lo(ww[e >> 1]);
-                const double df = (double)__bfloat162float(xv[j8 * 8 + e]) + 0.5 * (double)c2;
+              for (int e = 0; e < C; ++e) {
+                const int j = s2 * C + e;
+                const uint32_t cw = *reinterpret_cast<const uint32_t*>(bt + kmaj_off(k, j & ~1, SBO));
+                const float c2 = (j & 1) ? bf16_hi(cw) : bf16_lo(cw);
+                const float xf = __bfloat162float(
+                    *reinterpret_cast<const __nv_bfloat16*>(rw + raw_off(s2, row, gi * C + e)));
+                const double df = (double)xf + 0.5 * (double)c2;
                 d2 = fma(df, df, d2);
               }
-            }
             return d2;
           };
           double best = 1e300;
@@ -402,12 +450,12 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
           if (tie) code = bk;
         }
         tc_fence_before();
-        if (valid_row && ok) {
+        if (mine && valid_row && ok) {
           const int cn = coded_offset + (t0 + row - tok_begin);
           idx[idx_code_off(g, layer, blk, req, h, kvi, cn, span * NGC + gi)] = (uint8_t)code;
         }
-        named_sync(1 + set, kRows);     // the set's TMEM columns and A tile are free again
-        mma_phase ^= 1u;                // one completed phase of this set's barrier per group
+        named_sync(1 + set, kSetThreads);   // the set's TMEM columns, A tile and block minima are free again
+        mma_phase ^= 1u;                     // one completed phase of this set's barrier per group
         if (!ok) break;
       }
       if (__syncthreads_or(fail_s[0] | fail_s[1])) failed = true;
@@ -421,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
     }
   }
   if (failed && tid == 0) set_status(st, LVQ_ETIMEOUT);
-  if (failed && row == 0)   // a set whose MMA wait gave up lets it finish before TMEM is freed
+  if (failed && set_leader)   // a set whose MMA wait gave up lets it finish before TMEM is freed
     mbar_wait(smem_addr(&bars[kRawStages + set]), mma_phase, kWaitIters);
   tc_fence_before();
   __syncthreads();
@@ -432,7 +480,9 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
 
 }  // namespace tc
 
-bool encode_tc_supported(int G, int c) { return (G == 16 || G == 32) && (c == 4 || c == 8) && c < G; }
+// (G, c) = (32, 4) would need Tc = 8 raw steps per tile: its shared-memory plan does not fit one
+// CTA, so the direct-form encoder serves it
+bool encode_tc_supported(int G, int c) { return (G == 16 && (c == 4 || c == 8)) || (G == 32 && c == 8); }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda dependency)
 static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -461,7 +511,7 @@ static cudaError_t encode_tc_as(const Geo& g, int layer, int req, const __nv_bfl
   cuuint32_t box[3] = {tc::kSpan, tc::kTileTokens, (cuuint32_t)X::TC};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16*>(kv), dims, strides, box,
-                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
 
@@ -494,7 +544,7 @@ cudaError_t launch_encode_tc(const Geo& g, int layer, int req, const __nv_bfloat
   if (g.G == GG && g.c == CC)                                                                            \
     return encode_tc_as<GG, CC>(g, layer, req, kv, tok_stride, kv_tokens, tok_begin, n_tok, coded_offset, \
                                 cb, idx, st, s);
-  LVQ_ETC(16, 4) LVQ_ETC(16, 8) LVQ_ETC(32, 4) LVQ_ETC(32, 8)
+  LVQ_ETC(16, 4) LVQ_ETC(16, 8) LVQ_ETC(32, 8)
 #undef LVQ_ETC
   return cudaErrorInvalidValue;
 }
