@@ -57,7 +57,7 @@ struct Enc {
   static constexpr int RAW = TC * kTileTokens * kSpan * 2;
   static constexpr int OFF_B = 0;
   static constexpr int OFF_A = OFF_B + NGC * B_TILE;
-  static constexpr int OFF_RAW = OFF_A + NGC * A_TILE;
+  static constexpr int OFF_RAW = OFF_A + 2 * NGC * A_TILE;   // A slots: [tile parity][group]
   static constexpr int OFF_NMAX = OFF_RAW + kRawStages * RAW;
   static constexpr int OFF_BAR = OFF_NMAX + 16 * 4;
   static constexpr int OFF_BMIN = OFF_BAR + 8 * (kRawStages + 2);     // [2 sets][8 blocks][128 rows]
@@ -198,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
     fail_s[1] = 0;
   }
   // zero the A tiles once: the columns past G + 3 stay zero
-  for (int i = tid; i < NGC * X::A_TILE / 16; i += kThreads)
+  for (int i = tid; i < 2 * NGC * X::A_TILE / 16; i += kThreads)
     reinterpret_cast<uint4*>(At)[i] = make_uint4(0, 0, 0, 0);
   tc_fence_before();
   __syncthreads();
@@ -213,6 +213,48 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
   const int n_sets = 2 * g.nblk * g.H * n_spans;
   const int n_ranges = (n_tok + kItemTokens - 1) / kItemTokens;
   const long n_items = (long)n_sets * n_ranges;
+
+  // A row of this thread's token for group gib from a raw tile: element s*c+e =
+  // raw[s][row][gib*c+e].  Both threads of a row read it (for ||x||^2); each writes half of
+  // its 16-byte chunks.  Returns ||x||^2 of the joint vector.
+  auto build_a = [&](const unsigned char* src_tile, int gib, unsigned char* at) -> float {
+    uint32_t xw[G / 2];                  // the row's G elements, two per word
+#pragma unroll
+    for (int s2 = 0; s2 < TC; ++s2) {
+      const unsigned char* src = src_tile + raw_off(s2, row, gib * C);
+      if constexpr (C == 4) {
+        const uint2 w = *reinterpret_cast<const uint2*>(src);
+        xw[s2 * 2] = w.x;
+        xw[s2 * 2 + 1] = w.y;
+      } else {
+        const uint4 w = *reinterpret_cast<const uint4*>(src);
+        xw[s2 * 4] = w.x;
+        xw[s2 * 4 + 1] = w.y;
+        xw[s2 * 4 + 2] = w.z;
+        xw[s2 * 4 + 3] = w.w;
+      }
+    }
+    float x2 = 0.f;
+#pragma unroll
+    for (int q = 0; q < G / 2; ++q) {
+      const float lo = bf16_lo(xw[q]), hi = bf16_hi(xw[q]);
+      x2 = fmaf(lo, lo, x2);
+      x2 = fmaf(hi, hi, x2);
+    }
+#pragma unroll
+    for (int k8 = 0; k8 < G / 8; ++k8)
+      if ((k8 >= G / 16) == (hf == 1))
+        *reinterpret_cast<uint4*>(at + kmaj_off(row, k8 * 8, SBO)) =
+            make_uint4(xw[k8 * 4], xw[k8 * 4 + 1], xw[k8 * 4 + 2], xw[k8 * 4 + 3]);
+    if (hf == 1) {
+      const uint32_t one = 0x3f80u;   // bf16 1.0
+      *reinterpret_cast<uint4*>(at + kmaj_off(row, G, SBO)) = make_uint4(one | (one << 16), one, 0u, 0u);
+    }
+    fence_proxy_async();             // the tile is read by the tensor core (async proxy)
+    return x2;
+  };
+  bool prebuilt = false;            // the set's next A tile was built during the previous MMA
+  float xx_next = 0.f;
 
   uint32_t raw_phase = 0;   // bit s: parity of raw stage s
   uint32_t mma_phase = 0;
@@ -291,55 +333,39 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
       const unsigned char* rw = raw + stg * X::RAW;
       const bool valid_row = t0 + row < t_last;
 
-      // each set handles groups gi = set, set + 2, ...
+      // each set handles groups gi = set, set + 2, ...; the A tile of the set's next group is
+      // built while the current group's MMA runs (A slots alternate with the tile parity)
       for (int gi = set; gi < NGC; gi += 2) {
-        // A row: joint vector of token t0+row, group gi: element s*c+e = raw[s][row][gi*c+e].
-        // Both threads of a row read it (for ||x||^2); each writes half of its 16-byte chunks.
-        unsigned char* at = At + gi * X::A_TILE;
-        float xx = 0.f;
-        {
-          uint32_t xw[G / 2];                  // the row's G elements, two per word
-#pragma unroll
-          for (int s2 = 0; s2 < TC; ++s2) {
-            const unsigned char* src = rw + raw_off(s2, row, gi * C);
-            if constexpr (C == 4) {
-              const uint2 w = *reinterpret_cast<const uint2*>(src);
-              xw[s2 * 2] = w.x;
-              xw[s2 * 2 + 1] = w.y;
-            } else {
-              const uint4 w = *reinterpret_cast<const uint4*>(src);
-              xw[s2 * 4] = w.x;
-              xw[s2 * 4 + 1] = w.y;
-              xw[s2 * 4 + 2] = w.z;
-              xw[s2 * 4 + 3] = w.w;
-            }
-          }
-#pragma unroll
-          for (int q = 0; q < G / 2; ++q) {
-            const float lo = bf16_lo(xw[q]), hi = bf16_hi(xw[q]);
-            xx = fmaf(lo, lo, xx);
-            xx = fmaf(hi, hi, xx);
-          }
-#pragma unroll
-          for (int k8 = 0; k8 < G / 8; ++k8)
-            if ((k8 >= G / 16) == (hf == 1))
-              *reinterpret_cast<uint4*>(at + kmaj_off(row, k8 * 8, SBO)) =
-                  make_uint4(xw[k8 * 4], xw[k8 * 4 + 1], xw[k8 * 4 + 2], xw[k8 * 4 + 3]);
-          if (hf == 1) {
-            const uint32_t one = 0x3f80u;   // bf16 1.0
-            *reinterpret_cast<uint4*>(at + kmaj_off(row, G, SBO)) = make_uint4(one | (one << 16), one, 0u, 0u);
-          }
+        const int slot = gi + NGC * (tile_counter & 1);
+        float xx;
+        if (prebuilt) {
+          xx = xx_next;
+          prebuilt = false;
+        } else {
+          xx = build_a(rw, gi, At + slot * X::A_TILE);
         }
-        fence_proxy_async();
         tc_fence_before();
         named_sync(1 + set, kSetThreads);
         if (set_leader) {
           tc_fence_after();
-          const uint32_t a0 = smem_addr(at), b0 = smem_addr(Bt + gi * X::B_TILE);
+          const uint32_t a0 = smem_addr(At + slot * X::A_TILE), b0 = smem_addr(Bt + gi * X::B_TILE);
 #pragma unroll
           for (int ks = 0; ks < X::KSTEPS; ++ks)
             mma_bf16(tmem_set, smem_desc(a0 + ks * 256, SBO), smem_desc(b0 + ks * 256, SBO), kIdesc, ks > 0);
           mma_commit(smem_addr(&bars[kRawStages + set]));
+        }
+        if (gi + 2 < NGC) {
+          xx_next = build_a(rw, gi + 2, At + (slot + 2) * X::A_TILE);
+          prebuilt = true;
+        } else if (tl + 1 < n_tiles) {
+          // the set's first group of the next tile: its raw stage was requested two tiles ago
+          const int stg1 = (tile_counter + 1) % kRawStages;
+          if (mbar_wait(smem_addr(&bars[stg1]), (raw_phase >> stg1) & 1u, kWaitIters)) {
+            xx_next = build_a(raw + stg1 * X::RAW, set, At + (set + NGC * ((tile_counter + 1) & 1)) * X::A_TILE);
+            prebuilt = true;
+          } else {
+            fail_s[set] = 1;
+          }
         }
         // one warp of the set waits for the MMA; the barrier releases the others (no spinning)
         if ((tid % kSetThreads) < 32) {
@@ -454,10 +480,13 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
           const int cn = coded_offset + (t0 + row - tok_begin);
           idx[idx_code_off(g, layer, blk, req, h, kvi, cn, span * NGC + gi)] = (uint8_t)code;
         }
-        named_sync(1 + set, kSetThreads);   // the set's TMEM columns, A tile and block minima are free again
+        // no barrier here: the next group's first barrier (before its MMA) is reached by every
+        // thread of the set only after this epilogue, so the TMEM columns, block minima and
+        // masks are free by then
         mma_phase ^= 1u;                     // one completed phase of this set's barrier per group
         if (!ok) break;
       }
+      fence_proxy_async();   // this thread's reads of the raw stage before its refill by TMA
       if (__syncthreads_or(fail_s[0] | fail_s[1])) failed = true;
       // refill this raw stage with the tile two ahead
       if (tid == 0 && tl + 2 < n_tiles) {
