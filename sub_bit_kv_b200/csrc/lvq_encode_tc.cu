@@ -61,8 +61,8 @@ struct Enc {
   static constexpr int OFF_NMAX = OFF_RAW + kRawStages * RAW;
   static constexpr int OFF_BAR = OFF_NMAX + 16 * 4;
   static constexpr int OFF_BMIN = OFF_BAR + 8 * (kRawStages + 2);     // [2 sets][8 blocks][128 rows]
-  static constexpr int OFF_MASK = OFF_BMIN + 2 * (kEntries / 32) * kRows * 4;   // [2 sets][2 halves][128 rows]
-  static constexpr int OFF_TMEM = OFF_MASK + 2 * 2 * kRows * 4;
+  static constexpr int OFF_MASK = OFF_BMIN + 2 * (kEntries / 32) * kRows * 4;   // [2 sets][8 blocks][128 rows]
+  static constexpr int OFF_TMEM = OFF_MASK + 2 * (kEntries / 32) * kRows * 4;
   // + alignment slack; at least 120 KB so that one CTA (holding all of TMEM) fits per SM
   static constexpr int SMEM = (OFF_TMEM + 16 + 1024) > 120 * 1024 ? (OFF_TMEM + 16 + 1024) : 120 * 1024;
   static_assert(NGC == 2 || NGC == 4, "two MMA sets alternate over the item's groups");
@@ -116,23 +116,6 @@ __device__ inline void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_
 __device__ inline void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" :: "r"(bar)
                : "memory");
-}
-
-// 32 consecutive fp32 columns of this thread's TMEM lane
-__device__ inline void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
-        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
-        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // 64 consecutive fp32 columns of this thread's TMEM lane, issued without waiting
@@ -207,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
   const uint32_t tmem_set = tmem_base + (uint32_t)(set * 256);
   const uint32_t lane_addr = ((uint32_t)(32 * (warp & 3))) << 16;
   float* const bmin_set = bmin_s + set * (kEntries / 32) * kRows;     // [8 blocks][128 rows]
-  uint32_t* const mask_set = mask_s + set * 2 * kRows;                // [2 halves][128 rows]
+  uint32_t* const mask_set = mask_s + set * (kEntries / 32) * kRows;  // [8 blocks][128 rows]
 
   const int n_spans = g.d / kSpan;
   const int n_sets = 2 * g.nblk * g.H * n_spans;
@@ -253,7 +236,16 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
     fence_proxy_async();             // the tile is read by the tensor core (async proxy)
     return x2;
   };
-  bool prebuilt = false;            // the set's next A tile was built during the previous MMA
+  // the set's UMMA of group gib from A slot aslot into the set's TMEM columns (one thread)
+  auto issue_mma = [&](int aslot, int gib) {
+    const uint32_t a0 = smem_addr(At + aslot * X::A_TILE), b0 = smem_addr(Bt + gib * X::B_TILE);
+#pragma unroll
+    for (int ks = 0; ks < X::KSTEPS; ++ks)
+      mma_bf16(tmem_set, smem_desc(a0 + ks * 256, SBO), smem_desc(b0 + ks * 256, SBO), kIdesc, ks > 0);
+    mma_commit(smem_addr(&bars[kRawStages + set]));
+  };
+  bool issued = false;              // the set's next MMA was issued during the previous group
+  bool outstanding = false;         // an MMA of this set may still be running
   float xx_next = 0.f;
 
   uint32_t raw_phase = 0;   // bit s: parity of raw stage s
@@ -271,6 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
     const int t_first = tok_begin + range * kItemTokens;
     const int t_last = min(tok_begin + n_tok, t_first + kItemTokens);
     const int n_tiles = (t_last - t_first + kTileTokens - 1) / kTileTokens;
+    uint8_t* const idx_item = idx + idx_stream_off(g, layer, blk, req, h, kvi);
 
     // all MMAs of the previous item have completed (each set waited for its commits)
     __syncthreads();
@@ -333,36 +326,34 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
       const unsigned char* rw = raw + stg * X::RAW;
       const bool valid_row = t0 + row < t_last;
 
-      // each set handles groups gi = set, set + 2, ...; the A tile of the set's next group is
-      // built while the current group's MMA runs (A slots alternate with the tile parity)
+      // each set handles groups gi = set, set + 2, ...  The A tile of the set's next group is
+      // built while the current group's MMA runs (A slots alternate with the tile parity), and
+      // that next MMA is issued as soon as the current one's accumulator has been read.
       for (int gi = set; gi < NGC; gi += 2) {
         const int slot = gi + NGC * (tile_counter & 1);
         float xx;
-        if (prebuilt) {
+        if (issued) {
           xx = xx_next;
-          prebuilt = false;
+          issued = false;
         } else {
           xx = build_a(rw, gi, At + slot * X::A_TILE);
+          tc_fence_before();
+          named_sync(1 + set, kSetThreads);
+          if (set_leader) issue_mma(slot, gi);
+          outstanding = true;
         }
-        tc_fence_before();
-        named_sync(1 + set, kSetThreads);
-        if (set_leader) {
-          tc_fence_after();
-          const uint32_t a0 = smem_addr(At + slot * X::A_TILE), b0 = smem_addr(Bt + gi * X::B_TILE);
-#pragma unroll
-          for (int ks = 0; ks < X::KSTEPS; ++ks)
-            mma_bf16(tmem_set, smem_desc(a0 + ks * 256, SBO), smem_desc(b0 + ks * 256, SBO), kIdesc, ks > 0);
-          mma_commit(smem_addr(&bars[kRawStages + set]));
-        }
+        int next_slot = -1, next_gi = 0;
         if (gi + 2 < NGC) {
-          xx_next = build_a(rw, gi + 2, At + (slot + 2) * X::A_TILE);
-          prebuilt = true;
+          next_slot = slot + 2;
+          next_gi = gi + 2;
+          xx_next = build_a(rw, next_gi, At + next_slot * X::A_TILE);
         } else if (tl + 1 < n_tiles) {
           // the set's first group of the next tile: its raw stage was requested two tiles ago
           const int stg1 = (tile_counter + 1) % kRawStages;
           if (mbar_wait(smem_addr(&bars[stg1]), (raw_phase >> stg1) & 1u, kWaitIters)) {
-            xx_next = build_a(raw + stg1 * X::RAW, set, At + (set + NGC * ((tile_counter + 1) & 1)) * X::A_TILE);
-            prebuilt = true;
+            next_slot = set + NGC * ((tile_counter + 1) & 1);
+            next_gi = set;
+            xx_next = build_a(raw + stg1 * X::RAW, set, At + next_slot * X::A_TILE);
           } else {
             fail_s[set] = 1;
           }
@@ -378,11 +369,9 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
         // epilogue, one pass over this warp's half of the row (four 32-column blocks, two
         // 64-column loads): each block's minimum, and the block's columns within eps of that
         // minimum as a bit mask (bit 31 - i for column i).  Of the block holding the row
-        // minimum, that mask is exactly the row's candidates inside it; any other block whose
-        // minimum is within eps of the row minimum holds further candidates.
-        const float eps = ldexpf(xx + nmax_s[gi], -14);
-        float hbest = __int_as_float(0x7f800000);   // +inf
-        uint32_t hmask = 0u;                        // candidate mask of this half's best block
+        // minimum, that mask is exactly the row's candidates inside it; of any other block it
+        // holds every candidate of the row in that block (its minimum is not below the row's).
+        const float eps = (xx + nmax_s[gi]) * 0x1p-14f;
 #pragma unroll 1
         for (int q2 = 0; q2 < 2; ++q2) {
           uint32_t ra[64];
@@ -399,7 +388,6 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
             }
             m0 = fmin3(m0, __uint_as_float(r[30]), __uint_as_float(r[31]));
             const float bm = fminf(m0, m1);
-            bmin_set[(hf * 4 + q2 * 2 + b2) * kRows + row] = bm;
             // sign of (bm + eps) - v per column, shifted in: 1 = outside the window
             const float tb = bm + eps;
             const float2 t2 = make_float2(tb, tb), neg1 = make_float2(-1.f, -1.f);
@@ -410,15 +398,26 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
               sg = __funnelshift_l(__float_as_uint(e.x), sg, 1);
               sg = __funnelshift_l(__float_as_uint(e.y), sg, 1);
             }
-            if (bm < hbest) {                          // strict: the first block of equal minima
-              hbest = bm;
-              hmask = ~sg;
-            }
+            const int q = hf * 4 + q2 * 2 + b2;
+            bmin_set[q * kRows + row] = bm;
+            mask_set[q * kRows + row] = ~sg;
           }
         }
-        mask_set[hf * kRows + row] = hmask;
+        tc_fence_before();
         named_sync(1 + set, kSetThreads);      // also: every thread saw the MMA wait's outcome
         const bool ok = fail_s[set] == 0;      // uniform over the set
+        if (ok) outstanding = false;
+        mma_phase ^= 1u;                       // one completed phase of this set's barrier per group
+        // the accumulator has been read: start the next group's MMA (its A tile was completed by
+        // every thread of the set before the barrier above)
+        if (ok && next_slot >= 0) {
+          if (set_leader) {
+            tc_fence_after();
+            issue_mma(next_slot, next_gi);
+          }
+          issued = true;
+          outstanding = true;
+        }
         float bmin[kEntries / 32];
 #pragma unroll
         for (int q = 0; q < kEntries / 32; ++q) bmin[q] = bmin_set[q * kRows + row];
@@ -434,56 +433,41 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
         }
         const int wb = at_min ? __ffs(at_min) - 1 : 0;   // the first block holding the minimum
         const bool mine = (wb >> 2) == hf;     // this thread's half holds it: it owns the row
-        const uint32_t cm = mask_set[(wb >> 2) * kRows + row];
+        const uint32_t cm = mask_set[wb * kRows + row];
         int code = wb * 32 + __clz(cm);
-        const bool tie = mine && (__popc(cm) + __popc(bmask & ~(1u << wb)) > 1);
-        if (__any_sync(0xffffffffu, tie && valid_row)) {
-          // near-tie: exact fp64 direct-form distances of every candidate (the row's candidate
-          // blocks are read again, from either half), lowest index on ties
+        const bool tie = mine && valid_row && (__popc(cm) + __popc(bmask & ~(1u << wb)) > 1);
+        if (tie) {
+          // near-tie: exact fp64 direct-form distances of the candidates of every block within
+          // eps (the block masks are supersets of them), lowest index on ties
           const unsigned char* bt = Bt + gi * X::B_TILE;
-          auto dist = [&](int k) {           // sum_j (x_j - C_kj)^2 in fp64; the tile holds -2 C in bf16
-            double d2 = 0.0;
-#pragma unroll
-            for (int s2 = 0; s2 < TC; ++s2)
-#pragma unroll
-              for (int e = 0; e < C; ++e) {
-                const int j = s2 * C + e;
-                const uint32_t cw = *reinterpret_cast<const uint32_t*>(bt + kmaj_off(k, j & ~1, SBO));
-                const float c2 = (j & 1) ? bf16_hi(cw) : bf16_lo(cw);
-                const float xf = __bfloat162float(
-                    *reinterpret_cast<const __nv_bfloat16*>(rw + raw_off(s2, row, gi * C + e)));
-                const double df = (double)xf + 0.5 * (double)c2;
-                d2 = fma(df, df, d2);
-              }
-            return d2;
-          };
           double best = 1e300;
           int bk = kEntries;
-          for (uint32_t wm = __reduce_or_sync(0xffffffffu, tie ? bmask : 0u); wm; wm &= wm - 1u) {
+          for (uint32_t wm = bmask; wm; wm &= wm - 1u) {
             const int q = __ffs(wm) - 1;
-            float v[32];
-            tmem_ld32(tmem_set + lane_addr + q * 32, v);
-            uint32_t m = 0u;
+            for (uint32_t m = mask_set[q * kRows + row]; m; m &= m - 1u) {
+              const int k = q * 32 + 32 - __ffs(m);       // bit 31 - i holds column i
+              double d2 = 0.0;                           // sum_j (x_j - C_kj)^2; the tile holds -2 C
 #pragma unroll
-            for (int i = 0; i < 32; ++i) m |= (v[i] <= thr ? 1u : 0u) << i;
-            if (!tie || !((bmask >> q) & 1u)) m = 0u;
-            for (; m; m &= m - 1u) {
-              const int k = q * 32 + __ffs(m) - 1;
-              const double d2 = dist(k);
+              for (int s2 = 0; s2 < TC; ++s2)
+#pragma unroll
+                for (int e = 0; e < C; ++e) {
+                  const int j = s2 * C + e;
+                  const uint32_t cw = *reinterpret_cast<const uint32_t*>(bt + kmaj_off(k, j & ~1, SBO));
+                  const float c2 = (j & 1) ? bf16_hi(cw) : bf16_lo(cw);
+                  const float xf = __bfloat162float(
+                      *reinterpret_cast<const __nv_bfloat16*>(rw + raw_off(s2, row, gi * C + e)));
+                  const double df = (double)xf + 0.5 * (double)c2;
+                  d2 = fma(df, df, d2);
+                }
               if (d2 < best || (d2 == best && k < bk)) { best = d2; bk = k; }
             }
           }
-          if (tie) code = bk;
+          code = bk;
         }
-        tc_fence_before();
         if (mine && valid_row && ok) {
           const int cn = coded_offset + (t0 + row - tok_begin);
-          idx[idx_code_off(g, layer, blk, req, h, kvi, cn, span * NGC + gi)] = (uint8_t)code;
+          idx_item[(size_t)(cn >> 3) * g.page_bytes + (span * NGC + gi) * kPage + (cn & 7)] = (uint8_t)code;
         }
-        // no barrier here: the next group's first barrier (before its MMA) is reached by every
-        // thread of the set only after this epilogue, so the TMEM columns, block minima and
-        // masks are free by then
-        mma_phase ^= 1u;                     // one completed phase of this set's barrier per group
         if (!ok) break;
       }
       fence_proxy_async();   // this thread's reads of the raw stage before its refill by TMA
@@ -498,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
     }
   }
   if (failed && tid == 0) set_status(st, LVQ_ETIMEOUT);
-  if (failed && set_leader)   // a set whose MMA wait gave up lets it finish before TMEM is freed
+  if (failed && set_leader && outstanding)   // let a set's last MMA finish before TMEM is freed
     mbar_wait(smem_addr(&bars[kRawStages + set]), mma_phase, kWaitIters);
   tc_fence_before();
   __syncthreads();
