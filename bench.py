@@ -53,7 +53,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="lvq", choices=["lvq", "reference"])
     ap.add_argument("--splits", type=int, default=0, help="split count (0: choose)")
-    ap.add_argument("--workload", default=WORKLOAD, choices=["ouro14_g16_32k", "ouro14_g32_b32", "ouro14_tc2_64k"],
+    ap.add_argument("--workload", default=WORKLOAD, choices=["ouro14_g16_32k", "ouro14_g32_b32", "ouro14_tc2_64k", "ouro14_tc1_32k"],
                     help="decode workload (the headline line uses the default)")
     ap.add_argument("--no-encode", action="store_true", help="skip the prefill-encode measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)

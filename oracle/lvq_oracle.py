@@ -309,3 +309,59 @@ def page_encode(recent_k: np.ndarray, recent_v: np.ndarray, cb_k: np.ndarray, cb
     ck, _, _ = encode(recent_k[:, :page], cb_k, Tc, G)
     cv, _, _ = encode(recent_v[:, :page], cb_v, Tc, G)
     return ck, cv
+
+
+# ------------------------------------------------------------------ codebook construction
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to the nearest bf16 value (ties to even), returned as fp64.
+
+    bf16 keeps 8 significant bits and fp32's exponent range (normal values from
+    2^-126, subnormal steps of 2^-133).  The rounding is done once, from fp64,
+    by scaling each value so that one bf16 step is 1 and rounding to the
+    nearest integer with ties to even (numpy's rint); values past the largest
+    finite bf16 become infinite.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    out = np.zeros_like(x)
+    nz = (x != 0) & np.isfinite(x)
+    _, e = np.frexp(x[nz])                       # |x| = m * 2^e, m in [0.5, 1)
+    step_exp = np.maximum(e - 8, -133)           # exponent of one bf16 step at |x|
+    r = np.rint(np.ldexp(x[nz], -step_exp))      # ties to even
+    out[nz] = np.ldexp(r, step_exp)
+    out[~np.isfinite(x)] = x[~np.isfinite(x)]
+    big = np.abs(out) > np.ldexp(255.0, 120)     # largest finite bf16 = (2 - 2^-7) * 2^127
+    out[big] = np.sign(out[big]) * np.inf
+    return out
+
+
+def kmeans_update(X: np.ndarray, codes: np.ndarray, C: np.ndarray):
+    """Update step of one plain k-means (Lloyd) iteration.
+
+    X: [M][G] joint vectors, codes: [M] their nearest entries, C: [256][G] the
+    current entries.  Returns (C_new [256][G] fp64, counts [256]): entry k moves
+    to the mean of the vectors coded k; an entry no vector chose keeps its value.
+
+    [summary, "how it differs"]: codebooks are initialised by k-means over joint
+    vectors (Fisher-weighted there; the weights need a model's gradients, so this
+    is the unweighted form).  [summary, "premises and limits"]: k-means over the
+    calibration tokens is the first calibration stage.  The pages leave empty
+    entries open; keeping them is the plainest reading.
+    """
+    C_new = np.array(C, dtype=np.float64, copy=True)
+    counts = np.zeros(C.shape[0], dtype=np.int64)
+    for k in range(C.shape[0]):
+        members = X[codes == k]
+        counts[k] = members.shape[0]
+        if counts[k] > 0:
+            C_new[k] = members.sum(axis=0) / counts[k]
+    return C_new, counts
+
+
+def kmeans_step(X: np.ndarray, C: np.ndarray):
+    """One Lloyd iteration with bf16 entries: assignment by nearest entry (lowest
+    index on ties), then the update step, the new entries rounded to bf16 as the
+    codebooks are stored.  Returns (codes, C_new, counts)."""
+    codes, _, _ = nearest_entry(X, C)
+    C_new, counts = kmeans_update(X, codes, C)
+    return codes, round_bf16(C_new), counts

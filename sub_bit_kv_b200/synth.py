@@ -108,6 +108,11 @@ WORKLOADS = {
     "ouro14_tc2_64k": Workload("ouro14_tc2_64k", n_layers=24, n_kv_heads=16, n_q_heads=16,
                                head_dim=128, T=4, Tc=2, G=16, batch=8, n_sink=4, n_recent=256,
                                ctx=65536, key_outliers=True, gen_tokens=256),
+    # per-step coding (Tc = 1, c = G = 16) at the same 0.5 bits per element: the degenerate
+    # case without a loop axis, a per-step baseline beside the joint coding of ouro14_g16_32k
+    "ouro14_tc1_32k": Workload("ouro14_tc1_32k", n_layers=24, n_kv_heads=16, n_q_heads=16,
+                               head_dim=128, T=4, Tc=1, G=16, batch=1, n_sink=4, n_recent=128,
+                               ctx=32768, key_outliers=True),
 }
 
 

@@ -22,6 +22,18 @@ def test_decode_bytes_closed_form_32k():
     assert got == idx + slices + bf16 + qo == 36_610_112
 
 
+def test_decode_bytes_per_step_coding_reads_one_block():
+    """Tc = 1 (c = 16): a step reads only its own block's 8 code bytes per token, head and K/V."""
+    w = synth.WORKLOADS["ouro14_tc1_32k"]
+    coded, recent = 32636, 128
+    got = bench.decode_bytes_per_launch(w, _Lay(8), [coded], [recent])
+    idx = coded * 16 * 2 * 8
+    slices = 16 * 2 * 256 * 128 * 2
+    bf16 = (4 + 128) * 16 * 2 * 128 * 2
+    qo = 16 * 128 * (2 + 4) + 16 * 4
+    assert got == idx + slices + bf16 + qo
+
+
 def test_decode_bytes_batch_counts_slices_once():
     w = synth.WORKLOADS["ouro14_g32_b32"]
     one = bench.decode_bytes_per_launch(w, _Lay(16), [1000], [128])

@@ -22,6 +22,7 @@ def _n_sm():
     ("ouro14_g16_32k", [(0, 0), (0, 7), (0, 15)]),         # 32K context, batch 1, G=16 (c=4)
     ("ouro14_g32_b32", [(0, 3), (13, 9), (31, 15)]),       # 32 ragged requests, G=32 (c=8)
     ("ouro14_tc2_64k", [(0, 0), (5, 11), (7, 15)]),        # 64K context, batch 8, Tc=2 (two blocks)
+    ("ouro14_tc1_32k", [(0, 2), (0, 13)]),                 # 32K context, per-step coding (Tc=1, c=16)
 ])
 def test_decode_full_size_sampled(name, samples):
     w = synth.WORKLOADS[name]

@@ -131,7 +131,7 @@ def test_codebook_entries_reencode_to_own_index():
 
 # ----------------------------------------------------------------------------------- dequant
 
-@pytest.mark.parametrize("name", ["tiny", "ouro14_tc2_64k", "ouro14_g32_b32"])
+@pytest.mark.parametrize("name", ["tiny", "ouro14_tc2_64k", "ouro14_g32_b32", "ouro14_tc1_32k"])
 def test_dequantize_bit_exact(name):
     w = synth.WORKLOADS[name] if name == "tiny" else _reduced(name, n_layers=2, n_kv_heads=3, n_q_heads=3)
     case = Hl.build_case(w, layers=2, ctx=[w.n_sink + 300 + w.n_recent])
@@ -181,6 +181,7 @@ def test_decode_tiny_all_steps(ns):
     ("ouro14_g16_32k", [4 + 777 + 131], 5),                 # ragged tail, recent window of 131
     ("ouro14_g32_b32", [2000, 1437, 133, 4, 3, 600], 8),     # ragged batch, tiny contexts
     ("ouro14_tc2_64k", [3000, 2321], 16),
+    ("ouro14_tc1_32k", [4 + 901 + 128, 700], 8),             # per-step coding: Tc = 1, c = 16
 ])
 def test_decode_reduced_shapes(name, ctx, ns):
     w = _reduced(name, n_layers=2, n_kv_heads=2, n_q_heads=2)
@@ -269,7 +270,7 @@ def test_identical_codes_zero_key_share_uniform_attention():
 
 # ----------------------------------------------------------------------------------- page encode
 
-@pytest.mark.parametrize("name", ["ouro14_tc2_64k", "ouro14_g16_32k", "ouro14_g32_b32"])
+@pytest.mark.parametrize("name", ["ouro14_tc2_64k", "ouro14_g16_32k", "ouro14_g32_b32", "ouro14_tc1_32k"])
 def test_page_encode_matches_oracle_and_advances(name):
     """Requests 0 and 2 have a full recent window and are encoded (several due requests share
     each codebook read); request 1 is one token short and is left untouched."""

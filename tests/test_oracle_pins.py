@@ -300,6 +300,75 @@ def test_page_encode_equals_prefill_encode():
     assert (pk == full_k[:, 16:24]).all() and (pv == full_v[:, 16:24]).all()
 
 
+# ----------------------------------------------------------------------------- codebook construction
+
+def test_kmeans_hand_fixture():
+    fx = _golden("kmeans_tiny.json")
+    C = np.array(fx["codebook"])
+    X = np.array(fx["x"])
+    codes, C_new, counts = O.kmeans_step(X, C)
+    assert codes.tolist() == fx["codes"]
+    np.testing.assert_array_equal(C_new, fx["new_codebook"])
+    assert counts.tolist() == fx["counts"]
+
+
+def test_kmeans_update_matches_sklearn_one_lloyd_iteration():
+    """No empty entries here (scikit-learn relocates empty clusters, the oracle keeps them)."""
+    from sklearn.cluster import KMeans
+    rng = np.random.default_rng(11)
+    K, G = 16, 4
+    centers = rng.standard_normal((K, G)) * 6
+    X = np.concatenate([centers[k] + rng.standard_normal((40, G)) for k in range(K)])
+    C = centers + rng.standard_normal((K, G)) * 0.5
+    codes, _, _ = O.nearest_entry(X, C)
+    assert len(set(codes.tolist())) == K
+    C_new, counts = O.kmeans_update(X, codes, C)
+    km = KMeans(n_clusters=K, init=C, n_init=1, max_iter=1, algorithm="lloyd", tol=0.0).fit(X)
+    np.testing.assert_allclose(C_new, km.cluster_centers_, rtol=0, atol=1e-12)
+    assert counts.sum() == X.shape[0]
+
+
+def test_kmeans_update_never_raises_the_objective():
+    """Lloyd descent: the mean minimises each entry's sum of squares, and re-assigning to
+    the nearest entry can only lower it further."""
+    rng = np.random.default_rng(5)
+    X = rng.standard_normal((3000, 8))
+    C = X[rng.choice(3000, 64, replace=False)] + 0.1
+    def sse(C_):
+        _, d1, _ = O.nearest_entry(X, C_)
+        return d1.sum()
+    codes, _, _ = O.nearest_entry(X, C)
+    C_new, counts = O.kmeans_update(X, codes, C)
+    assert sse(C_new) <= sse(C)
+    # the update is the minimiser: moving any used entry a little raises its members' sum
+    k = int(np.argmax(counts))
+    m = X[codes == k]
+    base = ((m - C_new[k]) ** 2).sum()
+    for dv in np.eye(8) * 1e-3:
+        assert ((m - (C_new[k] + dv)) ** 2).sum() > base
+
+
+def test_kmeans_empty_entry_keeps_its_value():
+    C = np.array([[0.0, 0.0], [100.0, 100.0], [-3.0, 7.0]])
+    X = np.array([[0.5, 0.0], [0.0, 0.5]])
+    C_new, counts = O.kmeans_update(X, np.array([0, 0]), C)
+    np.testing.assert_array_equal(C_new[1:], C[1:])
+    assert counts.tolist() == [2, 0, 0]
+
+
+def test_round_bf16_matches_torch_on_fp32_values_and_ties_go_even():
+    rng = np.random.default_rng(2)
+    x = (rng.standard_normal(50000) * np.exp(rng.standard_normal(50000) * 8)).astype(np.float32)
+    ref = torch.tensor(x).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.round_bf16(x.astype(np.float64)), ref)
+    # halfway cases from fp64 (not representable in fp32 rounding twice): ties to even
+    assert O.round_bf16(np.array([1 + 2.0 ** -8]))[0] == 1.0
+    assert O.round_bf16(np.array([1 + 3 * 2.0 ** -8]))[0] == 1 + 2.0 ** -6
+    assert O.round_bf16(np.array([1 + 2.0 ** -8 + 2.0 ** -40]))[0] == 1 + 2.0 ** -7
+    assert O.round_bf16(np.array([2.0 ** -134]))[0] == 0.0          # half the smallest subnormal
+    assert O.round_bf16(np.array([2.0 ** 128]))[0] == np.inf
+
+
 # ----------------------------------------------------------------------------- planted mistakes
 
 def test_pins_catch_planted_mistakes(monkeypatch):
@@ -357,3 +426,43 @@ def test_pins_catch_planted_mistakes(monkeypatch):
         test_joint_vector_order_fixture()
     monkeypatch.undo()
     del O._dq_orig
+
+    def update_sum_not_mean(X, codes, C):       # forgets to divide by the count
+        C_new = np.array(C, dtype=np.float64, copy=True)
+        counts = np.zeros(C.shape[0], dtype=np.int64)
+        for k in range(C.shape[0]):
+            m = X[codes == k]
+            counts[k] = m.shape[0]
+            if counts[k]:
+                C_new[k] = m.sum(axis=0)
+        return C_new, counts
+
+    monkeypatch.setattr(O, "kmeans_update", update_sum_not_mean)
+    with pytest.raises(AssertionError):
+        test_kmeans_hand_fixture()
+    with pytest.raises(AssertionError):
+        test_kmeans_update_matches_sklearn_one_lloyd_iteration()
+    monkeypatch.undo()
+
+    def update_zeroes_empty(X, codes, C):      # empty entries collapse to the origin
+        C_new = np.zeros_like(np.asarray(C, dtype=np.float64))
+        counts = np.zeros(C.shape[0], dtype=np.int64)
+        for k in range(C.shape[0]):
+            m = X[codes == k]
+            counts[k] = m.shape[0]
+            if counts[k]:
+                C_new[k] = m.mean(axis=0)
+        return C_new, counts
+
+    monkeypatch.setattr(O, "kmeans_update", update_zeroes_empty)
+    with pytest.raises(AssertionError):
+        test_kmeans_empty_entry_keeps_its_value()
+    monkeypatch.undo()
+
+    def round_via_fp32(x):                      # double rounding fp64 -> fp32 -> bf16
+        return torch.tensor(np.asarray(x, dtype=np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+
+    monkeypatch.setattr(O, "round_bf16", round_via_fp32)
+    with pytest.raises(AssertionError):
+        test_round_bf16_matches_torch_on_fp32_values_and_ties_go_even()
+    monkeypatch.undo()
