@@ -462,6 +462,25 @@ def gpu_arm(args):
                "distance_gemm_tflops": tflops, "frac_of_bf16_peak": tflops / tpk, "bf16_peak": tpk,
                "peak_kind": tpk_kind,
                "workload": "ouro26_prefill_32k (one of 48 layers)", "kernel": "encode_tc (tcgen05 distance GEMM + argmin)"}
+        # codebook construction: the k-means update step over the codes the encoder just wrote
+        # (one Lloyd iteration = this encode + this update); it reads the layer's bf16 K/V and
+        # its codes once
+        argsk = (cfg4, c4.lay, 0, 0, kv4, 0, wc.ctx, 0, c4.idx, c4.cb, None, c4.status)
+        lvq.lvq_kmeans_update(*argsk)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(3):
+            lvq.lvq_kmeans_update(*argsk)
+        b_.record()
+        torch.cuda.synchronize()
+        c4.check_status("kmeans update")
+        upd_ms = a.elapsed_time(b_) / 3
+        upd_bytes = kv4.numel() * 2 + vectors + c4.lay.cb_bytes
+        enc["kmeans"] = {"update_ms": upd_ms, "iteration_ms": enc_ms + upd_ms,
+                         "iteration_vectors_per_s": vectors / ((enc_ms + upd_ms) / 1e3),
+                         "update_gbps": upd_bytes / (upd_ms / 1e3) / 1e9,
+                         "update_frac_of_hbm": upd_bytes / (upd_ms / 1e3) / 1e9 / peaks()[0],
+                         "kernel": "kmeans_update (fp64 shared-memory sums per entry)"}
         del kv4, c4
 
     if rank != 0:

@@ -176,6 +176,30 @@ LVQ_API lvq_status lvq_encode_prefill(const lvq_config* cfg, const lvq_layout* l
                               int32_t coded_offset, const void* cb, uint8_t* idx,
                               int32_t* dev_status, void* stream);
 
+/* Codebook construction: the update step of one plain k-means (Lloyd)
+ * iteration over the joint vectors of one layer ("LoopVQ summary", "how it
+ * differs": codebooks are initialised by k-means over joint vectors -- Fisher-
+ * weighted there, unweighted here; "premises and limits": k-means over the
+ * calibration tokens).  The assignment step is lvq_encode_prefill with the same
+ * layer, req, kv, tokens and coded_offset; this call then moves every entry of
+ * every (K/V, block, head, group) codebook of `layer` to the mean of the joint
+ * vectors coded with it (fp64 sums, the mean rounded once to bf16, to nearest,
+ * ties to even) and leaves an entry that no vector chose unchanged.
+ *   kv, kv_tok_stride, kv_tokens, tok_begin, n_tok, coded_offset: as for
+ *     lvq_encode_prefill (tokens [tok_begin, tok_begin + n_tok) of kv, their
+ *     codes in slots [coded_offset, coded_offset + n_tok) of request req).
+ *   idx: the code buffer holding those codes (read only).
+ *   cb: logical codebooks, updated in place for `layer` (lay->cb_*).
+ *   counts: nullable device uint32 [2][n_blk][Hkv][n_g][256]: vectors per entry.
+ * The packed codebooks and norms the decoder reads are not touched: call
+ * lvq_pack_codebooks after the last iteration.  LVQ_EUNSUPPORTED where
+ * (d/c) is not a multiple of 64/G. */
+LVQ_API lvq_status lvq_kmeans_update(const lvq_config* cfg, const lvq_layout* lay, int32_t layer,
+                             int32_t req, const void* kv, int64_t kv_tok_stride, int32_t kv_tokens,
+                             int32_t tok_begin, int32_t n_tok, int32_t coded_offset,
+                             const uint8_t* idx, void* cb, uint32_t* counts, int32_t* dev_status,
+                             void* stream);
+
 /* Decode-time page encode ("LoopVQ summary", "premises and limits": new tokens
  * go to the recent window; every 8 tokens the oldest page is quantized across
  * all layers and loop steps).  For every request b < batch whose recent

@@ -173,6 +173,29 @@ lvq_status lvq_encode_prefill(const lvq_config* cfg, const lvq_layout* lay, int3
                                            static_cast<cudaStream_t>(stream)));
 }
 
+lvq_status lvq_kmeans_update(const lvq_config* cfg, const lvq_layout* lay, int32_t layer, int32_t req,
+                             const void* kv, int64_t kv_tok_stride, int32_t kv_tokens, int32_t tok_begin,
+                             int32_t n_tok, int32_t coded_offset, const uint8_t* idx, void* cb, uint32_t* counts,
+                             int32_t* dev_status, void* stream) {
+  (void)dev_status;
+  Geo g;
+  lvq_status s = check_all(cfg, lay, &g);
+  if (s != LVQ_OK) return s;
+  if (layer < 0 || layer >= g.L || req < 0 || req >= g.B || n_tok < 0 || tok_begin < 0 ||
+      kv_tokens < 0 || (int64_t)tok_begin + n_tok > kv_tokens || coded_offset < 0 ||
+      (int64_t)coded_offset + n_tok > (int64_t)g.P * kPage || kv_tok_stride < (int64_t)g.H * g.d)
+    return LVQ_EINVAL;
+  if (!kv || !cb || !idx || !aligned16(kv) || !aligned16(cb) || !aligned16(idx) ||
+      (counts && !aligned16(counts)))
+    return LVQ_EINVAL;
+  if (g.ng % (64 / g.G) != 0) return LVQ_EUNSUPPORTED;
+  if ((s = check_device()) != LVQ_OK) return s;
+  return cuda_status(launch_kmeans_update(g, layer, req, static_cast<const __nv_bfloat16*>(kv), kv_tok_stride,
+                                          kv_tokens, tok_begin, n_tok, coded_offset, idx,
+                                          static_cast<__nv_bfloat16*>(cb), counts,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 lvq_status lvq_encode_page(const lvq_config* cfg, const lvq_layout* lay, int32_t batch, const int32_t* ctx_len,
                            int32_t* coded_len, const void* ring, const void* cb, const float* cb_norm,
                            uint8_t* idx, int32_t* dev_status, void* stream) {

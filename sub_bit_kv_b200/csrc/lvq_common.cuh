@@ -124,6 +124,9 @@ cudaError_t launch_encode_page(const Geo& g, int batch, const int32_t* ctx_len, 
                                const __nv_bfloat16* ring, const __nv_bfloat16* cb, const float* cb_norm,
                                uint8_t* idx, int32_t* st, cudaStream_t s);
 constexpr int kPageMaxBatch = 1024;     // requests one lvq_encode_page call can take
+cudaError_t launch_kmeans_update(const Geo& g, int layer, int req, const __nv_bfloat16* kv, int64_t tok_stride,
+                                 int kv_tokens, int tok_begin, int n_tok, int coded_offset, const uint8_t* idx,
+                                 __nv_bfloat16* cb, uint32_t* counts, cudaStream_t s);
 cudaError_t launch_decode(const Geo& g, int layer, int step, int batch, const __nv_bfloat16* q,
                           const int32_t* ctx_len, const int32_t* coded_len,
                           const __nv_bfloat16* sink, const __nv_bfloat16* ring, const uint8_t* idx,

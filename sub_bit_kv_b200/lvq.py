@@ -57,6 +57,8 @@ _SIGS = {
                              _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P, _P, _P],
     "lvq_dequantize": [ctypes.POINTER(lvq_config), ctypes.POINTER(lvq_layout), _I32, _I32, _I32, _I32, _P,
                        _P, _I32, _I32, _P, _P],
+    "lvq_kmeans_update": [ctypes.POINTER(lvq_config), ctypes.POINTER(lvq_layout), _I32, _I32, _P,
+                          ctypes.c_int64, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P],
     "lvq_status_string": [_I32],
     "lvq_decode_attention_noalloc": [ctypes.POINTER(lvq_config), ctypes.POINTER(lvq_layout), _I32, _I32, _I32,
                                      _P, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P, _P],
@@ -150,6 +152,24 @@ def lvq_encode_prefill(cfg, lay, layer, req, kv, tok_begin, n_tok, coded_offset,
         tok_begin, n_tok, coded_offset, _ptr(cb, "cb", torch.bfloat16, lay.cb_bytes),
         _ptr(idx, "idx", torch.uint8, lay.idx_bytes), _ptr(dev_status, "dev_status", torch.int32, 4),
         _stream(stream)), "lvq_encode_prefill")
+
+
+def lvq_kmeans_update(cfg, lay, layer, req, kv, tok_begin, n_tok, coded_offset, idx, cb, counts, dev_status,
+                      kv_tok_stride=None, stream=None):
+    """Update step of one k-means iteration after lvq_encode_prefill wrote the codes.
+    kv: bf16 [2][T][N][Hkv][d] of one layer and request (contiguous); cb is updated in
+    place; counts: None or int32 [2][n_blk][Hkv][n_g][256] (the library writes uint32)."""
+    if kv.dim() != 5 or kv.shape[0] != 2 or kv.shape[1] != cfg.T:
+        raise ValueError("kv must be [2][T][N][Hkv][d]")
+    n_total = kv.shape[2]
+    stride = kv_tok_stride if kv_tok_stride is not None else kv.shape[3] * kv.shape[4]
+    n_counts = 2 * lay.n_blocks * cfg.n_kv_heads * lay.n_groups * 256
+    _check(lib().lvq_kmeans_update(
+        ctypes.byref(cfg), ctypes.byref(lay), layer, req, _ptr(kv, "kv", torch.bfloat16), stride, n_total,
+        tok_begin, n_tok, coded_offset, _ptr(idx, "idx", torch.uint8, lay.idx_bytes),
+        _ptr(cb, "cb", torch.bfloat16, lay.cb_bytes),
+        _ptr(counts, "counts", torch.int32, 4 * n_counts, optional=True),
+        _ptr(dev_status, "dev_status", torch.int32, 4), _stream(stream)), "lvq_kmeans_update")
 
 
 def lvq_encode_page(cfg, lay, batch, ctx_len, coded_len, ring, cb, cb_norm, idx, dev_status, stream=None):
