@@ -57,7 +57,7 @@ def parse():
                     help="decode workload (the headline line uses the default)")
     ap.add_argument("--no-encode", action="store_true", help="skip the prefill-encode measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--profile", default="", choices=["", "decode", "encode"],
+    ap.add_argument("--profile", default="", choices=["", "decode", "encode", "kmeans"],
                     help="build the workload, run 3 launches of one kernel and exit (for ncu captures)")
     return ap.parse_args()
 
@@ -276,6 +276,21 @@ def decode_bytes_per_launch(w, lay, coded, recent) -> int:
     return total
 
 
+def profile_kmeans(lvq, synth, torch, device):
+    """One Ouro-2.6B-shaped layer (32768 tokens): one encode, then the k-means update 3 times."""
+    wc = synth.WORKLOADS["ouro26_prefill_32k"]
+    cfg4 = lvq.make_config(1, wc.n_kv_heads, wc.n_q_heads, wc.head_dim, wc.T, wc.Tc, wc.G, 0, 0, 1, wc.ctx,
+                           max_splits=1, rope_base=wc.rope_base)
+    c4 = lvq.CodedCache(cfg4, device)
+    c4.cb_view()[0] = synth.codebooks(wc, 0, device=device)
+    kv4 = synth.loop_kv(wc, 0, wc.ctx, stream="coded", device=device)
+    lvq.lvq_encode_prefill(cfg4, c4.lay, 0, 0, kv4, 0, wc.ctx, 0, c4.cb, c4.idx, c4.status)
+    for _ in range(3):
+        lvq.lvq_kmeans_update(cfg4, c4.lay, 0, 0, kv4, 0, wc.ctx, 0, c4.idx, c4.cb, None, c4.status)
+    torch.cuda.synchronize()
+    c4.check_status("profile kmeans")
+
+
 def profile_encode(lvq, synth, torch, device):
     """One Ouro-2.6B-shaped layer (32768 tokens), encoded 3 times."""
     wc = synth.WORKLOADS["ouro26_prefill_32k"]
@@ -311,6 +326,9 @@ def gpu_arm(args):
 
     if args.profile == "encode":
         profile_encode(lvq, synth, torch, device)
+        return
+    if args.profile == "kmeans":
+        profile_kmeans(lvq, synth, torch, device)
         return
     w = synth.WORKLOADS[args.workload]
     replays = 2 * args.steps + args.warmup + 3          # every graph replay adds 8 tokens

@@ -177,7 +177,6 @@ lvq_status lvq_kmeans_update(const lvq_config* cfg, const lvq_layout* lay, int32
                              const void* kv, int64_t kv_tok_stride, int32_t kv_tokens, int32_t tok_begin,
                              int32_t n_tok, int32_t coded_offset, const uint8_t* idx, void* cb, uint32_t* counts,
                              int32_t* dev_status, void* stream) {
-  (void)dev_status;
   Geo g;
   lvq_status s = check_all(cfg, lay, &g);
   if (s != LVQ_OK) return s;
@@ -188,11 +187,11 @@ lvq_status lvq_kmeans_update(const lvq_config* cfg, const lvq_layout* lay, int32
   if (!kv || !cb || !idx || !aligned16(kv) || !aligned16(cb) || !aligned16(idx) ||
       (counts && !aligned16(counts)))
     return LVQ_EINVAL;
-  if (g.ng % (64 / g.G) != 0) return LVQ_EUNSUPPORTED;
+  if (g.ng % (64 / g.G) != 0 || kv_tok_stride % 8 != 0) return LVQ_EUNSUPPORTED;
   if ((s = check_device()) != LVQ_OK) return s;
   return cuda_status(launch_kmeans_update(g, layer, req, static_cast<const __nv_bfloat16*>(kv), kv_tok_stride,
                                           kv_tokens, tok_begin, n_tok, coded_offset, idx,
-                                          static_cast<__nv_bfloat16*>(cb), counts,
+                                          static_cast<__nv_bfloat16*>(cb), counts, dev_status,
                                           static_cast<cudaStream_t>(stream)));
 }
 

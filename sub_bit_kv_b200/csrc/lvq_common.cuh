@@ -1,6 +1,8 @@
 // Internal definitions shared by liblvq's translation units (not installed).
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -104,6 +106,17 @@ __device__ inline uint32_t smem_addr(const void* p) {
 }
 
 constexpr long kWaitIters = 1L << 24;   // bound of every device-side wait
+
+// Tiled TMA load of a 3-D box into this CTA's shared memory, completing on `bar` (no
+// multicast; the innermost coordinate times the element size must be a multiple of 16).
+__device__ inline void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+      :: "r"(dst), "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar) : "memory");
+}
+
+// cuTensorMapEncodeTiled from the driver (through the runtime's entry-point query); null if absent
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 constexpr int kMaxDevices = 64;
 
 }  // namespace lvq
@@ -126,7 +139,7 @@ cudaError_t launch_encode_page(const Geo& g, int batch, const int32_t* ctx_len, 
 constexpr int kPageMaxBatch = 1024;     // requests one lvq_encode_page call can take
 cudaError_t launch_kmeans_update(const Geo& g, int layer, int req, const __nv_bfloat16* kv, int64_t tok_stride,
                                  int kv_tokens, int tok_begin, int n_tok, int coded_offset, const uint8_t* idx,
-                                 __nv_bfloat16* cb, uint32_t* counts, cudaStream_t s);
+                                 __nv_bfloat16* cb, uint32_t* counts, int32_t* st, cudaStream_t s);
 cudaError_t launch_decode(const Geo& g, int layer, int step, int batch, const __nv_bfloat16* q,
                           const int32_t* ctx_len, const int32_t* coded_len,
                           const __nv_bfloat16* sink, const __nv_bfloat16* ring, const uint8_t* idx,

@@ -28,9 +28,6 @@
 // issue its UMMA, and run the argmin epilogue, so one set's epilogue overlaps
 // the other set's MMA.  In a set, warps w and w + 4 read the same TMEM lane
 // quadrant (32 rows) and split the 256 entries into halves.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include "lvq_common.cuh"
 
 namespace lvq {
@@ -85,12 +82,6 @@ constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((256u >> 3) <<
 // byte offset of element (row, k) of a K-major no-swizzle tile
 __device__ inline uint32_t kmaj_off(int row, int k, int sbo) {
   return (row & 7) * 16 + (row >> 3) * sbo + (k >> 3) * 128 + (k & 7) * 2;
-}
-
-__device__ inline void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
-      :: "r"(dst), "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar) : "memory");
 }
 
 // byte offset of channel ch of token row r (of step s) in a raw tile written by TMA with
@@ -498,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
 bool encode_tc_supported(int G, int c) { return (G == 16 && (c == 4 || c == 8)) || (G == 32 && c == 8); }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda dependency)
-static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
     void* p = nullptr;
