@@ -193,7 +193,10 @@ LVQ_API lvq_status lvq_encode_prefill(const lvq_config* cfg, const lvq_layout* l
  *   counts: nullable device uint32 [2][n_blk][Hkv][n_g][256]: vectors per entry.
  * The packed codebooks and norms the decoder reads are not touched: call
  * lvq_pack_codebooks after the last iteration.  LVQ_EUNSUPPORTED where
- * (d/c) is not a multiple of 64/G. */
+ * (d/c) is not a multiple of 64/G or kv_tok_stride is not a multiple of 8
+ * (the values are read by TMA); LVQ_EINVAL for out-of-range arguments, null
+ * or misaligned (16-byte) pointers.  Device-side: LVQ_ETIMEOUT in *dev_status
+ * if a copy never lands (every wait is bounded). */
 LVQ_API lvq_status lvq_kmeans_update(const lvq_config* cfg, const lvq_layout* lay, int32_t layer,
                              int32_t req, const void* kv, int64_t kv_tok_stride, int32_t kv_tokens,
                              int32_t tok_begin, int32_t n_tok, int32_t coded_offset,
