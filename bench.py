@@ -65,8 +65,8 @@ def parse():
 # DRAM bytes (read + write) of one decode_kernel<128,4> launch of this workload, from one ncu
 # capture (`python bench.py --profile decode` under ncu), valid only for the decode source it was
 # taken on: the bench reports it when the file's hash still matches, else null.
-DECODE_TRAFFIC = {"source_sha256": "3ceba606b1e1a640ac4dcfa48f7d83a1a99ca28cb698ab3329f3e3acc9453ced",
-                  "bytes_per_launch": 36771712}
+DECODE_TRAFFIC = {"source_sha256": "e0a90d0177e361757c3c3bd8c0ee087efc08e819b2f2ef52106cad027a658191",
+                  "bytes_per_launch": 36770560}
 
 
 def decode_traffic():

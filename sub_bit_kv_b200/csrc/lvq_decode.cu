@@ -63,7 +63,10 @@ struct Dec {
   static constexpr int F = D / 2;          // RoPE frequencies
   static constexpr int NG = D / C;         // groups per step
   static constexpr int NP = NG / 2;        // pair-groups (groups g, g + NG/2)
-  static constexpr int TQ = 32 / NP;       // token phases of the score mapping
+  static constexpr int LS = C > 8 ? C / 8 : 1;   // score lanes per pair-group (8 frequencies at most each)
+  static constexpr int CL = C / LS;        // frequencies of one score lane
+  static constexpr int NPV = NP * LS;      // score lanes of one token phase
+  static constexpr int TQ = 32 / NPV;      // token phases of the score mapping
   static constexpr int TPL = kPage / TQ;   // score tokens per lane per page
   static constexpr int TPV = 32 / NG;      // lanes per group in the value phase
   static constexpr int VPL = kPage / TPV;  // value tokens per lane per page
@@ -87,7 +90,7 @@ struct Dec {
   static constexpr int NSC_FIT = (kSmemMax - OFF_SC) / 4 / kChunk;
   static constexpr int NSC = (NSC_FIT < kMaxSuperChunks ? NSC_FIT : kMaxSuperChunks) * kChunk;
   static constexpr int SMEM = OFF_SC + NSC * 4;
-  static_assert(NP >= 4 && NP <= 32 && 32 % NP == 0, "pair-group mapping");
+  static_assert(NPV >= 4 && NPV <= 32 && 32 % NPV == 0, "pair-group mapping");
   static_assert(NG >= 8 && NG <= 32 && 32 % NG == 0, "value mapping");
   static_assert((1 << SH) == NG * 4, "histogram row");
   static_assert(NSC >= kChunk && SMEM <= kSmemMax, "shared memory");
@@ -167,25 +170,37 @@ __device__ inline void load_row(const unsigned char* base, uint32_t off, uint32_
 // Per-lane state of the score mapping.
 template <int D, int C>
 struct Lane {
-  int P, tq;
-  uint32_t gb_lo, gb_hi;              // byte offsets of the lane's two groups inside a slice row
+  int vp, P, tq, f0;                  // lane in its token phase, pair-group, token phase, first frequency
+  uint32_t gb_lo, gb_hi;              // byte offsets of the lane's share of its two groups in a slice row
   uint32_t sel[2];
-  float2 twoc[C], mtwoc[C];           // (2 cos, 2 cos) and its negation, of the lane's token stride
+  float2 twoc[Dec<D, C>::CL], mtwoc[Dec<D, C>::CL];   // (2 cos, 2 cos) and its negation, token stride
 };
+
+// The score lane `lane` of a token phase covers frequencies [f0, f0 + CL): those of pair-group
+// P = vp / LS, share vp % LS.
+template <int D, int C>
+__device__ inline int lane_f0(int lane) {
+  using X = Dec<D, C>;
+  const int vp = lane % X::NPV;
+  return (vp / X::LS) * C + (vp % X::LS) * X::CL;
+}
 
 template <int D, int C>
 __device__ inline void lane_init(Lane<D, C>& L, int lane, const float2* etq_s) {
   using X = Dec<D, C>;
-  constexpr int NP = X::NP, TQ = X::TQ;
-  L.P = lane % NP;
-  L.tq = lane / NP;
-  L.gb_lo = (uint32_t)L.P * C * 2;
-  L.gb_hi = (uint32_t)(L.P + NP) * C * 2;
+  constexpr int NP = X::NP, TQ = X::TQ, CL = X::CL;
+  L.vp = lane % X::NPV;
+  L.P = L.vp / X::LS;
+  L.tq = lane / X::NPV;
+  L.f0 = lane_f0<D, C>(lane);
+  const uint32_t share = (uint32_t)(L.vp % X::LS) * CL * 2;
+  L.gb_lo = (uint32_t)L.P * C * 2 + share;
+  L.gb_hi = (uint32_t)(L.P + NP) * C * 2 + share;
   L.sel[0] = row_sel(L.tq);
   L.sel[1] = row_sel(L.tq + (TQ == 2 ? 2 : 0));
 #pragma unroll
-  for (int e = 0; e < C; ++e) {
-    const float cs = etq_s[L.P * C + e].x;          // cos(TQ theta_f)
+  for (int e = 0; e < CL; ++e) {
+    const float cs = etq_s[L.f0 + e].x;             // cos(TQ theta_f)
     L.twoc[e] = make_float2(2.f * cs, 2.f * cs);
     L.mtwoc[e] = make_float2(-2.f * cs, -2.f * cs);
   }
@@ -204,11 +219,11 @@ __device__ inline void lane_init(Lane<D, C>& L, int lane, const float2* etq_s) {
 // NP tokens.
 template <int D, int C>
 __device__ inline float run_scores(const Lane<D, C>& L, const unsigned char* Ks, const unsigned char* pages,
-                                   float2 (&Wc)[C], float2 (&Wn)[C]) {
+                                   float2 (&Wc)[Dec<D, C>::CL], float2 (&Wn)[Dec<D, C>::CL]) {
   using X = Dec<D, C>;
-  constexpr int TQ = X::TQ, TPL = X::TPL, NP = X::NP;
-  static_assert(kPPW * TPL == NP, "one token per lane after the reduction");
-  float acc[NP];
+  constexpr int TQ = X::TQ, TPL = X::TPL, NP = X::NP, NPV = X::NPV, CL = X::CL;
+  static_assert(kPPW * TPL == NPV, "one token per lane after the reduction");
+  float acc[NPV];
 #pragma unroll
   for (int pi = 0; pi < kPPW; ++pi) {
     const unsigned char* pg = pages + pi * X::PAGE;
@@ -228,29 +243,29 @@ __device__ inline float run_scores(const Lane<D, C>& L, const unsigned char* Ks,
         xh = word ? whi.y : whi.x;
         sel = L.sel[(TQ * i / 2) & 1];
       }
-      uint32_t lo[C / 2], hi[C / 2];
-      load_row<C>(Ks, row_addr<D>(xl, L.gb_lo, sel), lo);
-      load_row<C>(Ks, row_addr<D>(xh, L.gb_hi, sel), hi);
+      uint32_t lo[CL / 2], hi[CL / 2];
+      load_row<CL>(Ks, row_addr<D>(xl, L.gb_lo, sel), lo);
+      load_row<CL>(Ks, row_addr<D>(xh, L.gb_hi, sel), hi);
       float2 a2 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int w = 0; w < C / 2; ++w) {
+      for (int w = 0; w < CL / 2; ++w) {
         a2 = __ffma2_rn(Wc[2 * w], make_float2(bf16_lo(lo[w]), bf16_lo(hi[w])), a2);
         a2 = __ffma2_rn(Wc[2 * w + 1], make_float2(bf16_hi(lo[w]), bf16_hi(hi[w])), a2);
       }
       acc[n] = (n & 2) ? -a2.x - a2.y : a2.x + a2.y;
 #pragma unroll
-      for (int e = 0; e < C; ++e) {
+      for (int e = 0; e < CL; ++e) {
         const float2 nx = __ffma2_rn((n & 1) ? L.twoc[e] : L.mtwoc[e], Wn[e], Wc[e]);
         Wc[e] = Wn[e];
         Wn[e] = nx;
       }
     }
   }
-  // transposed reduction over the NP lanes of a token phase: at each level a lane
-  // keeps the half of its values selected by bit o of P and adds its partner's
+  // transposed reduction over the NPV lanes of a token phase: at each level a lane
+  // keeps the half of its values selected by bit o of vp and adds its partner's
 #pragma unroll
-  for (int o = NP / 2; o > 0; o >>= 1) {
-    const bool up = (L.P & o) != 0;
+  for (int o = NPV / 2; o > 0; o >>= 1) {
+    const bool up = (L.vp & o) != 0;
 #pragma unroll
     for (int k = 0; k < o; ++k) {
       const float send = up ? acc[k] : acc[k + o];
@@ -552,11 +567,12 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
     for (int ci = 0; ci < min(kStages, n_stream); ++ci) issue_chunk(ci);
   // a compute lane's RoPE factors at its first coded token, fetched now so that their latency
   // overlaps the prologue
-  float2 rf[C];
+  float2 rf[X::CL];
   if (!producer && do_coded) {
-    const int p_first = g.S + n0 + kPage * kPPW * warp + lane / X::NP;
+    const int p_first = g.S + n0 + kPage * kPPW * warp + lane / X::NPV;
+    const int f0 = lane_f0<D, C>(lane);
 #pragma unroll
-    for (int e = 0; e < C; ++e) rf[e] = rope_at(rope, g.RC, F, p_first, (lane % X::NP) * C + e);
+    for (int e = 0; e < X::CL; ++e) rf[e] = rope_at(rope, g.RC, F, p_first, f0 + e);
   }
   if (!bad && tid < F) {
     const __nv_bfloat16* qv = q + ((size_t)b * g.Hq + hq) * D;
@@ -610,10 +626,10 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
       // ---- compute warps
       Lane<D, C> L;
       lane_init<D, C>(L, lane, etq_s);
-      float2 U[C];                       // W of the lane's first token of the current chunk
+      float2 U[X::CL];                   // W of the lane's first token of the current chunk
 #pragma unroll
-      for (int e = 0; e < C; ++e) U[e] = cmul(zq[L.P * C + e], cconj(rf[e]));
-      const int pi_own = L.P / X::TPL, t_own = L.tq + TQ * (L.P % X::TPL);   // the lane's token of a run
+      for (int e = 0; e < X::CL; ++e) U[e] = cmul(zq[L.f0 + e], cconj(rf[e]));
+      const int pi_own = L.vp / X::TPL, t_own = L.tq + TQ * (L.vp % X::TPL);   // the lane's token of a run
       const int gv = lane % NG, tp = lane / NG;
       const uint32_t hl = smem_addr(Hs) + (uint32_t)gv * 4;
       uint32_t* PW = reinterpret_cast<uint32_t*>(SC);
@@ -632,11 +648,11 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
           if (!timed_out) {
             const int c0 = s0 + kc * kChunk;
             const unsigned char* stage = ringb + (ci % kStages) * X::STAGE;
-            float2 Wc[C], Wn[C];
+            float2 Wc[X::CL], Wn[X::CL];
 #pragma unroll
-            for (int e = 0; e < C; ++e) {
+            for (int e = 0; e < X::CL; ++e) {
               Wc[e] = U[e];
-              Wn[e] = cmul(U[e], etq_s[L.P * C + e]);     // s_1 = +1
+              Wn[e] = cmul(U[e], etq_s[L.f0 + e]);        // s_1 = +1
             }
             // pages past the split's end hold stale codes: their tokens are masked
             const float sc_ = run_scores<D, C>(L, Ks, stage + warp * kPPW * X::PAGE, Wc, Wn);
@@ -648,7 +664,7 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
             if (lane == 0) mbar_arrive(smem_addr(&bars[2 + kStages + ci % kStages]));
           }
 #pragma unroll
-          for (int e = 0; e < C; ++e) U[e] = cmul(U[e], ech_s[L.P * C + e]);
+          for (int e = 0; e < X::CL; ++e) U[e] = cmul(U[e], ech_s[L.f0 + e]);
         }
         // ---- weights: exact maximum, then integers round(2^(s - M) * 2^k) with 2^k * sum < 2^30
         mx = warp_max(mx);
