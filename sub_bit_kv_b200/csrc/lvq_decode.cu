@@ -63,7 +63,7 @@ struct Dec {
   static constexpr int F = D / 2;          // RoPE frequencies
   static constexpr int NG = D / C;         // groups per step
   static constexpr int NP = NG / 2;        // pair-groups (groups g, g + NG/2)
-  static constexpr int LS = C > 8 ? C / 8 : 1;   // score lanes per pair-group (8 frequencies at most each)
+  static constexpr int LS = C > 4 ? C / 4 : 1;   // score lanes per pair-group (4 frequencies each)
   static constexpr int CL = C / LS;        // frequencies of one score lane
   static constexpr int NPV = NP * LS;      // score lanes of one token phase
   static constexpr int TQ = 32 / NPV;      // token phases of the score mapping
