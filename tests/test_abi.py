@@ -103,3 +103,28 @@ def test_layout_mismatch_is_rejected_before_any_device_work():
     st = lvq.lib().lvq_decode_attention(ctypes.byref(cfg), ctypes.byref(lay), 0, 4, 1, *([None] * 8), 1,
                                         None, None, None, None, None, None)
     assert st == lvq.LVQ_EINVAL          # step 4 out of range for T = 4
+
+
+def test_kmeans_update_argument_checks_on_the_host():
+    """lvq_kmeans_update rejects bad arguments before any device work (no GPU needed)."""
+    import ctypes
+    w = synth.WORKLOADS["tiny"]
+    cfg = make_cfg(w)
+    lay = lvq.lvq_cache_layout(cfg)
+    L = lvq.lib()
+    fake = 1 << 20                       # a 16-byte-aligned address that is never touched
+
+    def call(layer=0, req=0, kv=fake, stride=w.n_kv_heads * w.head_dim, kv_tokens=64, tok_begin=0, n_tok=64,
+             coded_offset=0, idx=fake, cb=fake, counts=None):
+        return L.lvq_kmeans_update(ctypes.byref(cfg), ctypes.byref(lay), layer, req, kv, stride, kv_tokens,
+                                   tok_begin, n_tok, coded_offset, idx, cb, counts, None, None)
+
+    assert call(layer=cfg.n_layers) == lvq.LVQ_EINVAL
+    assert call(req=cfg.max_batch) == lvq.LVQ_EINVAL
+    assert call(n_tok=65) == lvq.LVQ_EINVAL                 # past the K/V buffer's tokens
+    assert call(kv=None) == lvq.LVQ_EINVAL
+    assert call(cb=fake + 8) == lvq.LVQ_EINVAL              # misaligned codebooks
+    assert call(stride=w.n_kv_heads * w.head_dim - 1) == lvq.LVQ_EINVAL
+    assert call(stride=w.n_kv_heads * w.head_dim + 4) == lvq.LVQ_EUNSUPPORTED   # rows TMA cannot read
+    big = lay.idx_bytes                                      # coded slots past the capacity
+    assert call(coded_offset=big) == lvq.LVQ_EINVAL
