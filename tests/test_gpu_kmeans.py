@@ -88,6 +88,34 @@ def test_kmeans_iteration_matches_oracle(name, ntok, extra):
     np.testing.assert_array_equal(cb_new[..., 7, :], cbo[..., 7, :])
 
 
+def test_kmeans_offsets_and_ragged_tail():
+    """Tokens taken from inside the K/V buffer (tok_begin = 5) and coded at an offset that is
+    not a page boundary (coded_offset = 3), with a ragged last tile: the update reads the same
+    vectors and codes the encoder used."""
+    w = _reduced("ouro14_g16_32k", n_layers=1, n_kv_heads=1, n_q_heads=1)
+    ntok, tb, co = 1000, 5, 3
+    case = Hl.build_case(w, layers=1, ctx=[w.n_sink + co + ntok + w.n_recent], coded=[co + ntok],
+                         codes_from="none")
+    c, cfg = case.cache, case.cfg
+    cb_old = case.cb[0].clone()
+    kv = synth.loop_kv(w, 0, tb + ntok + 7, stream="kmeans").cuda()
+    counts = torch.zeros(2 * c.lay.n_blocks * cfg.n_kv_heads * c.lay.n_groups * 256, dtype=torch.int32,
+                         device="cuda")
+    lvq.lvq_encode_prefill(cfg, c.lay, 0, 0, kv, tb, ntok, co, c.cb, c.idx, c.status)
+    lvq.lvq_kmeans_update(cfg, c.lay, 0, 0, kv, tb, ntok, co, c.idx, c.cb, counts, c.status)
+    torch.cuda.synchronize()
+    c.check_status()
+    counts = counts.view(2, c.lay.n_blocks, cfg.n_kv_heads, c.lay.n_groups, 256).cpu().numpy()
+    cb_new = Hl.f64(c.cb_view()[0].cpu())
+    codes_gpu = [Hl.get_codes(c, 0, 0, kvi, co, ntok).numpy() for kvi in range(2)]
+    x = Hl.f64(kv.cpu()[:, :, tb:tb + ntok])
+    cbo = Hl.f64(cb_old)
+    for kvi in range(2):
+        for g in range(c.lay.n_groups):
+            _compare(w, cbo, cb_new, counts, codes_gpu, x, kvi, 0, 0, g)
+    assert counts.sum() == 2 * c.lay.n_groups * ntok
+
+
 def test_kmeans_two_iterations_lower_the_objective():
     """Lloyd descent on the GPU path: the second iteration's codes fit at least as well."""
     w = _reduced("ouro14_g16_32k", n_layers=1, n_kv_heads=1, n_q_heads=1)
