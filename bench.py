@@ -36,6 +36,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -160,7 +161,10 @@ class Clocks:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        # the raw samples go to $LVQ_CLOCKS_DIR (default: the temporary directory); the JSON
+        # line carries their summary
+        out_dir = os.environ.get("LVQ_CLOCKS_DIR", tempfile.gettempdir())
+        self.path = os.path.join(out_dir, f"lvq_clocks_rank{index}_{os.getpid()}.csv")
 
     def __enter__(self):
         try:
