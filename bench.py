@@ -58,6 +58,8 @@ def parse():
                     help="decode workload (the headline line uses the default)")
     ap.add_argument("--no-encode", action="store_true", help="skip the prefill-encode measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-sample", type=int, default=2,
+                    help="single-head attentions per step of the reference (oracle) arm")
     ap.add_argument("--profile", default="", choices=["", "decode", "encode", "kmeans"],
                     help="build the workload, run 3 launches of one kernel and exit (for ncu captures)")
     return ap.parse_args()
@@ -97,57 +99,87 @@ def bf16_peak():
 
 # ------------------------------------------------------------------------------ oracle baseline
 
-def cpu_baseline(seconds: float):
-    """Times the fp64 oracle on whole head-attentions of the workload (32K context)."""
-    import numpy as np
+class _OracleDecode:
+    """The fp64 oracle on single-head decode attentions of the headline workload (32K
+    context, 1 thread): inputs built once, then any number of head-attentions timed."""
+
+    def __init__(self):
+        import numpy as np  # noqa: F401
+        from oracle import lvq_oracle as O
+        from sub_bit_kv_b200 import synth
+        self.O, self.synth = O, synth
+        w = self.w = synth.WORKLOADS[WORKLOAD]
+        L = w.ctx - w.n_sink - w.n_recent
+        f = lambda t: t.to(dtype=__import__("torch").float64).numpy()
+        self.cbf = f(synth.codebooks(w, 0))
+        self.skf = f(synth.loop_kv(w, 0, w.n_sink, stream="sink"))
+        self.rkf = f(synth.loop_kv(w, 0, w.n_recent, stream="recent"))
+        self.codes = synth.random_codes((2, 1, L, w.n_groups), seed=7).numpy()
+        self.n = 0
+        self.per_token = w.n_layers * w.T * w.n_q_heads          # head-attentions per decode token
+
+    def run(self, count: int) -> float:
+        """Runs `count` head-attentions; returns the elapsed seconds."""
+        w, O, cbf, skf, rkf = self.w, self.O, self.cbf, self.skf, self.rkf
+        t0 = time.perf_counter()
+        for _ in range(count):
+            h, step = self.n % w.n_kv_heads, self.n % w.T
+            q = self.synth.queries(w, 0, step)[0, h].to(dtype=__import__("torch").float64).numpy()
+            O.decode_attention(q, step, w.Tc, w.G, skf[0, step, :, h], skf[1, step, :, h], self.codes[0],
+                               self.codes[1], cbf[0, :, h], cbf[1, :, h], rkf[0, step, :, h], rkf[1, step, :, h],
+                               base=w.rope_base)
+            self.n += 1
+        return time.perf_counter() - t0
+
+
+def _one_thread():
     try:
         from threadpoolctl import threadpool_limits
-        limiter = threadpool_limits(limits=1)
+        return threadpool_limits(limits=1)
     except Exception:  # pragma: no cover
-        limiter = None
-    from oracle import lvq_oracle as O
-    from sub_bit_kv_b200 import synth
+        return None
 
-    w = synth.WORKLOADS[WORKLOAD]
-    L = w.ctx - w.n_sink - w.n_recent
-    cb = synth.codebooks(w, 0)
-    sk = synth.loop_kv(w, 0, w.n_sink, stream="sink")
-    rk = synth.loop_kv(w, 0, w.n_recent, stream="recent")
-    codes = synth.random_codes((2, 1, L, w.n_groups), seed=7)
-    f = lambda t: t.to(dtype=__import__("torch").float64).numpy()
-    cbf, skf, rkf = f(cb), f(sk), f(rk)
-    n, t0 = 0, time.perf_counter()
-    while True:
-        h, step = n % w.n_kv_heads, n % w.T
-        q = f(synth.queries(w, 0, step)[0, h])
-        O.decode_attention(q, step, w.Tc, w.G, skf[0, step, :, h], skf[1, step, :, h], codes[0].numpy(),
-                           codes[1].numpy(), cbf[0, :, h], cbf[1, :, h], rkf[0, step, :, h], rkf[1, step, :, h],
-                           base=w.rope_base)
+
+def cpu_baseline(seconds: float):
+    """Times the fp64 oracle on whole head-attentions of the workload (32K context) for
+    about `seconds`."""
+    limiter = _one_thread()
+    od = _OracleDecode()
+    n, el = 0, 0.0
+    while el < seconds:
+        el += od.run(1)
         n += 1
-        el = time.perf_counter() - t0
-        if el >= seconds:
-            break
     if limiter is not None:
         limiter.unregister()
-    per_token = w.n_layers * w.T * w.n_q_heads          # head-attentions per decode token
-    tok_s = n / el / per_token
-    return {"value": tok_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} single-head decode attentions at {w.ctx} context (fp64 numpy, 1 thread), "
-                      f"scaled by {per_token} head-attentions per token"}
+    return {"value": n / el / od.per_token, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} single-head decode attentions at {od.w.ctx} context (fp64 numpy, 1 thread), "
+                      f"scaled by {od.per_token} head-attentions per token"}
 
 
 def reference_arm(args):
+    """The oracle on the host: W untimed steps, then K timed steps, each step a bounded sample
+    of the workload (args.ref_sample single-head attentions, scaled to decode tokens)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    cb = cpu_baseline(args.cpu_seconds)
-    line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tokens/s",
+    limiter = _one_thread()
+    od = _OracleDecode()
+    for _ in range(args.warmup):
+        od.run(args.ref_sample)
+    el = sum(od.run(args.ref_sample) for _ in range(args.steps))
+    if limiter is not None:
+        limiter.unregister()
+    value = args.steps * args.ref_sample / el / od.per_token
+    cb = {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+          "sample": f"{args.steps} steps of {args.ref_sample} single-head decode attentions at {od.w.ctx} "
+                    f"context (fp64 numpy, 1 thread), scaled by {od.per_token} head-attentions per token"}
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": TOKENS_PER_STEP / cb["value"] * 1e3, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": TOKENS_PER_STEP / value * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD, "global_batch": 1, "seq_len": 32768, "parallelism": "cpu"},
             "cpu_baseline": cb,
-            "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
