@@ -142,6 +142,15 @@ LVQ_API lvq_status lvq_cache_layout(const lvq_config* cfg, lvq_layout* out);
 /* Message for a status code (static string, never NULL). */
 LVQ_API const char* lvq_status_string(lvq_status s);
 
+/* Test hook, not for normal use (process-global; not thread-safe).  Every device-side wait
+ * of the later calls gives up after `wait_iters` polls (<= 0: the normal bound, about 2^24)
+ * and reports LVQ_ETIMEOUT in *dev_status; `fault_mask` makes a copy never happen, so that
+ * such a wait runs out: bit 0 -- lvq_decode_attention skips the first code chunk of every
+ * CTA; bit 1 -- lvq_kmeans_update skips the first tile of every CTA.  Kernels still wait
+ * (bounded) for every copy they did issue before they exit, so the context stays usable.
+ * LVQ_EINVAL for unknown bits.  lvq_debug_faults(0, 0) restores normal operation. */
+LVQ_API lvq_status lvq_debug_faults(int64_t wait_iters, int32_t fault_mask);
+
 /* Helper: packs the logical codebooks (cb, see lvq_layout.cb_*) into the
  * step-major layout the decoder reads (cbp) and computes each entry's squared
  * norm in fp64, rounded to fp32 (cb_norm, may be NULL).  All device

@@ -30,6 +30,10 @@ lvq_status check_cfg(const lvq_config* c) {
   return LVQ_OK;
 }
 
+// test hook state (lvq_debug_faults); the defaults leave every kernel as in normal use
+static long debug_wait_iters = kWaitIters;
+static int debug_fault = 0;
+
 Geo make_geo(const lvq_config* c) {
   Geo g;
   g.L = c->n_layers; g.H = c->n_kv_heads; g.Hq = c->n_q_heads; g.d = c->head_dim;
@@ -40,6 +44,8 @@ Geo make_geo(const lvq_config* c) {
   g.B = c->max_batch; g.max_ctx = c->max_ctx; g.max_splits = c->max_splits;
   g.RC = max((c->max_ctx + kPage - 1) / kPage, 64) + 16;   // rows cover offsets up to 512 positions
   g.page_bytes = g.ng * kPage;
+  g.wait_iters = debug_wait_iters;
+  g.fault = debug_fault;
   return g;
 }
 
@@ -253,6 +259,14 @@ lvq_status lvq_dequantize(const lvq_config* cfg, const lvq_layout* lay, int32_t 
   return cuda_status(launch_dequantize(g, layer, step, req, kv, idx, static_cast<const __nv_bfloat16*>(cbp),
                                        tok_begin, n_tok, static_cast<__nv_bfloat16*>(out),
                                        static_cast<cudaStream_t>(stream)));
+}
+
+
+lvq_status lvq_debug_faults(int64_t wait_iters, int32_t fault_mask) {
+  if (fault_mask & ~(kFaultDecodeDropChunk | kFaultKmeansDropTile)) return LVQ_EINVAL;
+  debug_wait_iters = wait_iters > 0 ? (long)wait_iters : kWaitIters;
+  debug_fault = fault_mask;
+  return LVQ_OK;
 }
 
 }  // extern "C"

@@ -19,7 +19,13 @@ struct Geo {
   int L, H, Hq, d, T, Tc, G, c, ng, nblk;
   int S, W, R, P, B, max_ctx, max_splits, RC;
   int page_bytes;
+  long wait_iters;   // bound of every device-side wait (kWaitIters unless a test lowers it)
+  int fault;         // test hook: kFault* bits, 0 in normal use
 };
+// Test hook bits (lvq_debug_faults): a copy that is never issued, so that a bounded wait
+// runs out and the kernel reports LVQ_ETIMEOUT.
+constexpr int kFaultDecodeDropChunk = 1;   // decode: the first code chunk of every CTA
+constexpr int kFaultKmeansDropTile = 2;    // k-means update: the first tile of every CTA
 
 // byte offset of the code stream [page][n_g][8] of (layer, blk, b, h, kv)
 __host__ __device__ inline size_t idx_stream_off(const Geo& g, int layer, int blk, int b, int h, int kv) {

@@ -396,7 +396,7 @@ __device__ bool bf16_share(Service& service, const Geo& g, int layer, int step, 
     }
     {
       bool done = false;
-      for (long it = 0; it < kWaitIters && !done; ++it) {
+      for (long it = 0; it < g.wait_iters && !done; ++it) {
         done = __all_sync(0xffffffffu, mbar_test(bar, batch & 1));
         if (!done) service();
       }
@@ -548,6 +548,7 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
   };
   // chunk `ci` of the stream: its first coded token and which half of the page stream it reads
   auto issue_chunk = [&](int ci) {
+    if ((g.fault & kFaultDecodeDropChunk) && ci == 0) return;   // test hook: this copy never happens
     const int sc = ci / (2 * CPS), r = ci % (2 * CPS);
     const int nk = min(CPS, n_kchunks - sc * CPS);
     const bool is_v = r >= nk;
@@ -614,7 +615,7 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
       if (lane == 0) {
         int ci = ci_next;
         for (; ci < n_stream; ++ci) {
-          if (!mbar_wait(smem_addr(&bars[2 + kStages + ci % kStages]), (ci / kStages - 1) & 1, kWaitIters)) {
+          if (!mbar_wait(smem_addr(&bars[2 + kStages + ci % kStages]), (ci / kStages - 1) & 1, g.wait_iters)) {
             timed_out = true;
             break;
           }
@@ -634,7 +635,7 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
       const uint32_t hl = smem_addr(Hs) + (uint32_t)gv * 4;
       uint32_t* PW = reinterpret_cast<uint32_t*>(SC);
       // waits are bounded; their outcome is made uniform over the warp, then over the compute warps
-      timed_out = __any_sync(0xffffffffu, !mbar_wait(smem_addr(&bars[0]), 0, kWaitIters));
+      timed_out = __any_sync(0xffffffffu, !mbar_wait(smem_addr(&bars[0]), 0, g.wait_iters));
       int ci = 0;
       for (int sc = 0; sc < n_super; ++sc) {
         const int s0 = n0 + sc * X::NSC, s1 = min(n1, s0 + X::NSC);
@@ -644,7 +645,7 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
         for (int kc = 0; kc < nk; ++kc, ++ci) {
           if (!timed_out)
             timed_out = __any_sync(0xffffffffu, !mbar_wait(smem_addr(&bars[2 + ci % kStages]), (ci / kStages) & 1,
-                                                           kWaitIters));
+                                                           g.wait_iters));
           if (!timed_out) {
             const int c0 = s0 + kc * kChunk;
             const unsigned char* stage = ringb + (ci % kStages) * X::STAGE;
@@ -710,7 +711,7 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
         for (int kc = 0; kc < nk; ++kc, ++ci) {
           if (!timed_out)
             timed_out = __any_sync(0xffffffffu, !mbar_wait(smem_addr(&bars[2 + ci % kStages]), (ci / kStages) & 1,
-                                                           kWaitIters));
+                                                           g.wait_iters));
           if (timed_out) continue;
           const int c0 = s0 + kc * kChunk;
           const unsigned char* stage = ringb + (ci % kStages) * X::STAGE;
@@ -725,7 +726,7 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
           if (lane == 0) mbar_arrive(smem_addr(&bars[2 + kStages + ci % kStages]));
         }
         if (!timed_out && sc == 0)
-          timed_out = __any_sync(0xffffffffu, !mbar_wait(smem_addr(&bars[1]), 0, kWaitIters));
+          timed_out = __any_sync(0xffffffffu, !mbar_wait(smem_addr(&bars[1]), 0, g.wait_iters));
         timed_out = compute_sync_or(timed_out);
         // ---- contraction: o[ch] = sum_a H[a][ch / c] * V[a][ch], two channels per thread
         const int cp = tid % NPAIR, rep = tid / NPAIR;
@@ -768,19 +769,19 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
     timed_out = bf16_share<D, C>(no_service, g, layer, step, b, h, j, ns, S_eff, Lc, nbj, sink, ring, rope, zq,
                                  smem + X::OFF_V, smem_addr(&bars[2 + 2 * kStages]), part_bf16, misc);
   // the key slice copy was issued by every CTA: let it land before the CTA can exit
-  if (tid == 0 && !do_coded && !mbar_wait(smem_addr(&bars[0]), 0, kWaitIters)) timed_out = true;
+  if (tid == 0 && !do_coded && !mbar_wait(smem_addr(&bars[0]), 0, g.wait_iters)) timed_out = true;
   if (__syncthreads_or(timed_out)) {
     if (tid == 0) {
       set_status(st, LVQ_ETIMEOUT);
-      mbar_wait(smem_addr(&bars[0]), 0, kWaitIters);
+      mbar_wait(smem_addr(&bars[0]), 0, g.wait_iters);
       misc[0] = 1;
       if (do_coded) {   // let every issued copy land before the CTA can exit
         const int issued = max(misc[2], min(kStages, n_stream));
-        if (misc[3]) mbar_wait(smem_addr(&bars[1]), 0, kWaitIters);
+        if (misc[3]) mbar_wait(smem_addr(&bars[1]), 0, g.wait_iters);
         for (int ci = max(0, issued - kStages); ci < issued; ++ci)
-          mbar_wait(smem_addr(&bars[2 + ci % kStages]), (ci / kStages) & 1, kWaitIters);
+          mbar_wait(smem_addr(&bars[2 + ci % kStages]), (ci / kStages) & 1, g.wait_iters);
       }
-      if (misc[4] > 0) mbar_wait(smem_addr(&bars[2 + 2 * kStages]), (misc[4] - 1) & 1, kWaitIters);
+      if (misc[4] > 0) mbar_wait(smem_addr(&bars[2 + 2 * kStages]), (misc[4] - 1) & 1, g.wait_iters);
     }
     __syncthreads();
   }

@@ -203,12 +203,12 @@ __global__ void __launch_bounds__(PageEnc<G, C>::NW * 32, 1) encode_page_kernel(
     if (c >= n_cb) break;
     const int slot = (int)(it % NBUF);
     if (lane == 0 && c + (NBUF - 1) * stride < n_cb) issue(c + (NBUF - 1) * stride, (int)((it + NBUF - 1) % NBUF));
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_addr(&wbar[slot]), (uint32_t)((it / NBUF) & 1), kWaitIters));
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_addr(&wbar[slot]), (uint32_t)((it / NBUF) & 1), g.wait_iters));
     if (!ok) {
       if (lane == 0) {
         set_status(st, LVQ_ETIMEOUT);
         for (long j = it; j < it + NBUF && first + j * stride < n_cb; ++j)   // copies still in flight
-          mbar_wait(smem_addr(&wbar[j % NBUF]), (uint32_t)((j / NBUF) & 1), kWaitIters);
+          mbar_wait(smem_addr(&wbar[j % NBUF]), (uint32_t)((j / NBUF) & 1), g.wait_iters);
       }
       break;
     }

@@ -309,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
     for (int tl = 0; tl < n_tiles && !failed; ++tl, ++tile_counter) {
       const int stg = tile_counter % kRawStages;
       const int t0 = t_first + tl * kTileTokens;
-      if (__syncthreads_or(!mbar_wait(smem_addr(&bars[stg]), (raw_phase >> stg) & 1u, kWaitIters))) {
+      if (__syncthreads_or(!mbar_wait(smem_addr(&bars[stg]), (raw_phase >> stg) & 1u, g.wait_iters))) {
         failed = true;
         break;
       }
@@ -341,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
         } else if (tl + 1 < n_tiles) {
           // the set's first group of the next tile: its raw stage was requested two tiles ago
           const int stg1 = (tile_counter + 1) % kRawStages;
-          if (mbar_wait(smem_addr(&bars[stg1]), (raw_phase >> stg1) & 1u, kWaitIters)) {
+          if (mbar_wait(smem_addr(&bars[stg1]), (raw_phase >> stg1) & 1u, g.wait_iters)) {
             next_slot = set + NGC * ((tile_counter + 1) & 1);
             next_gi = set;
             xx_next = build_a(raw + stg1 * X::RAW, set, At + next_slot * X::A_TILE);
@@ -352,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
         // one warp of the set waits for the MMA; the barrier releases the others (no spinning)
         if ((tid % kSetThreads) < 32) {
           __syncwarp();
-          if (!mbar_wait(smem_addr(&bars[kRawStages + set]), mma_phase, kWaitIters)) fail_s[set] = 1;
+          if (!mbar_wait(smem_addr(&bars[kRawStages + set]), mma_phase, g.wait_iters)) fail_s[set] = 1;
         }
         named_sync(1 + set, kSetThreads);
         tc_fence_after();
@@ -474,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
   }
   if (failed && tid == 0) set_status(st, LVQ_ETIMEOUT);
   if (failed && set_leader && outstanding)   // let a set's last MMA finish before TMEM is freed
-    mbar_wait(smem_addr(&bars[kRawStages + set]), mma_phase, kWaitIters);
+    mbar_wait(smem_addr(&bars[kRawStages + set]), mma_phase, g.wait_iters);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

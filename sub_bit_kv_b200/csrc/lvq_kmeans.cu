@@ -103,6 +103,7 @@ __global__ void __launch_bounds__(kThreads, 1) kmeans_update_kernel(
   __syncthreads();
 
   auto issue = [&](int tl) {             // one thread: the tile's values and code pages
+    if ((g.fault & kFaultKmeansDropTile) && tl == 0) return;   // test hook: this copy never happens
     unsigned char* stg = smem + X::OFF_STAGE + (tl % kStages) * X::STAGE;
     const uint32_t bar = smem_addr(&bars[tl % kStages]);
     mbar_expect_tx(bar, X::RAW + X::CODES);
@@ -129,7 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1) kmeans_update_kernel(
   int tl = 0;
   for (; tl < n_tiles; ++tl) {
     const unsigned char* stg = smem + X::OFF_STAGE + (tl % kStages) * X::STAGE;
-    if (__syncthreads_or(!mbar_wait(smem_addr(&bars[tl % kStages]), (tl / kStages) & 1u, kWaitIters))) {
+    if (__syncthreads_or(!mbar_wait(smem_addr(&bars[tl % kStages]), (tl / kStages) & 1u, g.wait_iters))) {
       failed = true;
       break;
     }
@@ -158,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1) kmeans_update_kernel(
     if (tid == 0) {
       set_status(st, LVQ_ETIMEOUT);
       for (int t2 = tl; t2 < min(n_tiles, tl + kStages); ++t2)
-        mbar_wait(smem_addr(&bars[t2 % kStages]), (t2 / kStages) & 1u, kWaitIters);
+        mbar_wait(smem_addr(&bars[t2 % kStages]), (t2 / kStages) & 1u, g.wait_iters);
     }
     __syncthreads();
     return;

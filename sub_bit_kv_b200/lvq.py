@@ -60,6 +60,7 @@ _SIGS = {
     "lvq_kmeans_update": [ctypes.POINTER(lvq_config), ctypes.POINTER(lvq_layout), _I32, _I32, _P,
                           ctypes.c_int64, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P],
     "lvq_status_string": [_I32],
+    "lvq_debug_faults": [ctypes.c_int64, _I32],
     "lvq_decode_attention_noalloc": [ctypes.POINTER(lvq_config), ctypes.POINTER(lvq_layout), _I32, _I32, _I32,
                                      _P, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P, _P],
 }
@@ -170,6 +171,12 @@ def lvq_kmeans_update(cfg, lay, layer, req, kv, tok_begin, n_tok, coded_offset, 
         _ptr(cb, "cb", torch.bfloat16, lay.cb_bytes),
         _ptr(counts, "counts", torch.int32, 4 * n_counts, optional=True),
         _ptr(dev_status, "dev_status", torch.int32, 4), _stream(stream)), "lvq_kmeans_update")
+
+
+def lvq_debug_faults(wait_iters: int = 0, fault_mask: int = 0):
+    """Test hook: bound of every device-side wait (0: the normal bound) and copies that never
+    happen (bit 0: decode's first code chunk, bit 1: k-means' first tile).  Process-global."""
+    _check(lib().lvq_debug_faults(int(wait_iters), int(fault_mask)), "lvq_debug_faults")
 
 
 def lvq_encode_page(cfg, lay, batch, ctx_len, coded_len, ring, cb, cb_norm, idx, dev_status, stream=None):

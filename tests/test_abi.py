@@ -128,3 +128,12 @@ def test_kmeans_update_argument_checks_on_the_host():
     assert call(stride=w.n_kv_heads * w.head_dim + 4) == lvq.LVQ_EUNSUPPORTED   # rows TMA cannot read
     big = lay.idx_bytes                                      # coded slots past the capacity
     assert call(coded_offset=big) == lvq.LVQ_EINVAL
+
+
+def test_debug_fault_hook_host_side():
+    """The failure-detection test hook checks its bits on the host and restores cleanly."""
+    with pytest.raises(lvq.LvqError) as e:
+        lvq.lvq_debug_faults(0, 1 << 5)
+    assert e.value.status == lvq.LVQ_EINVAL
+    lvq.lvq_debug_faults(1 << 10, 3)
+    lvq.lvq_debug_faults(0, 0)
