@@ -68,8 +68,8 @@ def parse():
 # DRAM bytes (read + write) of one decode_kernel<128,4> launch of this workload, from one ncu
 # capture (`python bench.py --profile decode` under ncu), valid only for the decode source it was
 # taken on: the bench reports it when the file's hash still matches, else null.
-DECODE_TRAFFIC = {"source_sha256": "72697b4d9b6eca2db4ebc5ba85298742f105db860969558af3baf553a597e037",
-                  "bytes_per_launch": 36772992}
+DECODE_TRAFFIC = {"source_sha256": "e9422eb0c0c52da9d84373c6bdacf44bd53c0350259b6b29ed0d4d54ef5ada21",
+                  "bytes_per_launch": 36771200}
 
 
 def decode_traffic():

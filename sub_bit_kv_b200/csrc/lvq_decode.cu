@@ -360,7 +360,7 @@ template <int D, int C, class Service>
 __device__ bool bf16_share(Service& service, const Geo& g, int layer, int step, int b, int h, int j, int ns, int S_eff, int Lc,
                            int nbj, const __nv_bfloat16* __restrict__ sink, const __nv_bfloat16* __restrict__ ring,
                            const float* __restrict__ rope, const float2* zq, unsigned char* area, uint32_t bar,
-                           float* part, int* misc) {
+                           float* part, int* misc, long wait_iters) {
   constexpr int F = D / 2, FPL = F / 32, CPL = D / 32, BB = kBf16Batch;
   static_assert(8 * F * 8 + BB * (F * 8 + 4 * D) <= kEntries * D * 2, "bf16 batch fits the value-slice area");
   const int lane = threadIdx.x & 31;
@@ -396,7 +396,7 @@ __device__ bool bf16_share(Service& service, const Geo& g, int layer, int step, 
     }
     {
       bool done = false;
-      for (long it = 0; it < g.wait_iters && !done; ++it) {
+      for (long it = 0; it < wait_iters && !done; ++it) {
         done = __all_sync(0xffffffffu, mbar_test(bar, batch & 1));
         if (!done) service();
       }
@@ -463,7 +463,9 @@ __device__ bool bf16_share(Service& service, const Geo& g, int layer, int step, 
   return to;
 }
 
-template <int D, int C>
+// DBG: the instantiation used while the test hook is active (its wait bound and fault bits
+// come from the geometry); the normal one keeps the constant bound.
+template <int D, int C, bool DBG>
 __global__ void __launch_bounds__(kThr, 1) decode_kernel(
     Geo g, int layer, int step, const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ ctx_len,
     const int32_t* __restrict__ coded_len, const __nv_bfloat16* __restrict__ sink,
@@ -472,6 +474,7 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
     float* __restrict__ ws, float* __restrict__ out, float* __restrict__ lse, float* __restrict__ split_lse,
     int32_t* st) {
   using X = Dec<D, C>;
+  const long wit = DBG ? g.wait_iters : kWaitIters;   // bound of every wait
   constexpr int F = X::F, NG = X::NG, TQ = X::TQ, NPAIR = X::NPAIR, NREP = X::NREP;
   extern __shared__ __align__(1024) unsigned char smem[];
   unsigned char* Ks = smem;
@@ -548,7 +551,7 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
   };
   // chunk `ci` of the stream: its first coded token and which half of the page stream it reads
   auto issue_chunk = [&](int ci) {
-    if ((g.fault & kFaultDecodeDropChunk) && ci == 0) return;   // test hook: this copy never happens
+    if (DBG && (g.fault & kFaultDecodeDropChunk) && ci == 0) return;   // test hook: this copy never happens
     const int sc = ci / (2 * CPS), r = ci % (2 * CPS);
     const int nk = min(CPS, n_kchunks - sc * CPS);
     const bool is_v = r >= nk;
@@ -607,7 +610,7 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
             issue_chunk(ci_next++);
       };
       timed_out = bf16_share<D, C>(service, g, layer, step, b, h, j, ns, S_eff, Lc, nbj, sink, ring, rope, zq,
-                                   smem + X::OFF_V, smem_addr(&bars[2 + 2 * kStages]), part_bf16, misc);
+                                   smem + X::OFF_V, smem_addr(&bars[2 + 2 * kStages]), part_bf16, misc, wit);
       if (lane == 0 && !timed_out) {
         issue_v_slice();
         misc[3] = 1;
@@ -615,7 +618,7 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
       if (lane == 0) {
         int ci = ci_next;
         for (; ci < n_stream; ++ci) {
-          if (!mbar_wait(smem_addr(&bars[2 + kStages + ci % kStages]), (ci / kStages - 1) & 1, g.wait_iters)) {
+          if (!mbar_wait(smem_addr(&bars[2 + kStages + ci % kStages]), (ci / kStages - 1) & 1, wit)) {
             timed_out = true;
             break;
           }
@@ -635,7 +638,7 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
       const uint32_t hl = smem_addr(Hs) + (uint32_t)gv * 4;
       uint32_t* PW = reinterpret_cast<uint32_t*>(SC);
       // waits are bounded; their outcome is made uniform over the warp, then over the compute warps
-      timed_out = __any_sync(0xffffffffu, !mbar_wait(smem_addr(&bars[0]), 0, g.wait_iters));
+      timed_out = __any_sync(0xffffffffu, !mbar_wait(smem_addr(&bars[0]), 0, wit));
       int ci = 0;
       for (int sc = 0; sc < n_super; ++sc) {
         const int s0 = n0 + sc * X::NSC, s1 = min(n1, s0 + X::NSC);
@@ -645,7 +648,7 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
         for (int kc = 0; kc < nk; ++kc, ++ci) {
           if (!timed_out)
             timed_out = __any_sync(0xffffffffu, !mbar_wait(smem_addr(&bars[2 + ci % kStages]), (ci / kStages) & 1,
-                                                           g.wait_iters));
+                                                           wit));
           if (!timed_out) {
             const int c0 = s0 + kc * kChunk;
             const unsigned char* stage = ringb + (ci % kStages) * X::STAGE;
@@ -711,7 +714,7 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
         for (int kc = 0; kc < nk; ++kc, ++ci) {
           if (!timed_out)
             timed_out = __any_sync(0xffffffffu, !mbar_wait(smem_addr(&bars[2 + ci % kStages]), (ci / kStages) & 1,
-                                                           g.wait_iters));
+                                                           wit));
           if (timed_out) continue;
           const int c0 = s0 + kc * kChunk;
           const unsigned char* stage = ringb + (ci % kStages) * X::STAGE;
@@ -726,7 +729,7 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
           if (lane == 0) mbar_arrive(smem_addr(&bars[2 + kStages + ci % kStages]));
         }
         if (!timed_out && sc == 0)
-          timed_out = __any_sync(0xffffffffu, !mbar_wait(smem_addr(&bars[1]), 0, g.wait_iters));
+          timed_out = __any_sync(0xffffffffu, !mbar_wait(smem_addr(&bars[1]), 0, wit));
         timed_out = compute_sync_or(timed_out);
         // ---- contraction: o[ch] = sum_a H[a][ch / c] * V[a][ch], two channels per thread
         const int cp = tid % NPAIR, rep = tid / NPAIR;
@@ -767,21 +770,21 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
   auto no_service = []() {};
   if (!do_coded && producer)
     timed_out = bf16_share<D, C>(no_service, g, layer, step, b, h, j, ns, S_eff, Lc, nbj, sink, ring, rope, zq,
-                                 smem + X::OFF_V, smem_addr(&bars[2 + 2 * kStages]), part_bf16, misc);
+                                 smem + X::OFF_V, smem_addr(&bars[2 + 2 * kStages]), part_bf16, misc, wit);
   // the key slice copy was issued by every CTA: let it land before the CTA can exit
-  if (tid == 0 && !do_coded && !mbar_wait(smem_addr(&bars[0]), 0, g.wait_iters)) timed_out = true;
+  if (tid == 0 && !do_coded && !mbar_wait(smem_addr(&bars[0]), 0, wit)) timed_out = true;
   if (__syncthreads_or(timed_out)) {
     if (tid == 0) {
       set_status(st, LVQ_ETIMEOUT);
-      mbar_wait(smem_addr(&bars[0]), 0, g.wait_iters);
+      mbar_wait(smem_addr(&bars[0]), 0, wit);
       misc[0] = 1;
       if (do_coded) {   // let every issued copy land before the CTA can exit
         const int issued = max(misc[2], min(kStages, n_stream));
-        if (misc[3]) mbar_wait(smem_addr(&bars[1]), 0, g.wait_iters);
+        if (misc[3]) mbar_wait(smem_addr(&bars[1]), 0, wit);
         for (int ci = max(0, issued - kStages); ci < issued; ++ci)
-          mbar_wait(smem_addr(&bars[2 + ci % kStages]), (ci / kStages) & 1, g.wait_iters);
+          mbar_wait(smem_addr(&bars[2 + ci % kStages]), (ci / kStages) & 1, wit);
       }
-      if (misc[4] > 0) mbar_wait(smem_addr(&bars[2 + 2 * kStages]), (misc[4] - 1) & 1, g.wait_iters);
+      if (misc[4] > 0) mbar_wait(smem_addr(&bars[2 + 2 * kStages]), (misc[4] - 1) & 1, wit);
     }
     __syncthreads();
   }
@@ -895,11 +898,15 @@ static cudaError_t decode_as(const Geo& g, int layer, int step, int batch, const
   cudaError_t ge = cudaGetDevice(&dev);
   if (ge != cudaSuccess) return ge;
   if (dev < 0 || dev >= kMaxDevices || !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, C, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Dec<D, C>::SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(decode_kernel<D, C, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Dec<D, C>::SMEM);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < kMaxDevices) attr_set[dev] = true;
   }
+  const bool dbg = g.fault != 0 || g.wait_iters != kWaitIters;   // the test hook is active
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3(ns, g.Hq, batch);
   lc.blockDim = dim3(kThr, 1, 1);
@@ -910,8 +917,11 @@ static cudaError_t decode_as(const Geo& g, int layer, int step, int batch, const
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = 1;
-  return cudaLaunchKernelEx(&lc, decode_kernel<D, C>, g, layer, step, q, ctx_len, coded_len, sink, ring, idx, cbp,
-                            rope, ns, ws, out, lse, split_lse, st);
+  if (dbg)
+    return cudaLaunchKernelEx(&lc, decode_kernel<D, C, true>, g, layer, step, q, ctx_len, coded_len, sink, ring,
+                              idx, cbp, rope, ns, ws, out, lse, split_lse, st);
+  return cudaLaunchKernelEx(&lc, decode_kernel<D, C, false>, g, layer, step, q, ctx_len, coded_len, sink, ring, idx,
+                            cbp, rope, ns, ws, out, lse, split_lse, st);
 }
 
 // Sink + recent-window tokens one call can take: a CTA keeps the scores of its
