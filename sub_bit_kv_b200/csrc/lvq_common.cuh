@@ -66,7 +66,6 @@ __device__ inline void set_status(int32_t* st, int code) {
 
 __device__ inline float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ inline float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-__device__ inline float bf16_at(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
 // Bounded spin on an mbarrier phase.  Returns false if the wait gave up.
 __device__ inline bool mbar_wait(uint32_t bar, uint32_t parity, long max_iter) {

@@ -34,6 +34,17 @@ def test_decode_bytes_per_step_coding_reads_one_block():
     assert got == idx + slices + bf16 + qo
 
 
+def test_decode_bytes_two_blocks_read_only_this_steps_block():
+    """Tc = 2 (c = 8): two index rows per token, a step reads the 16 bytes of its own block."""
+    w = synth.WORKLOADS["ouro14_tc2_64k"]
+    got = bench.decode_bytes_per_launch(w, _Lay(16), [65276], [256])
+    idx = 65276 * 16 * 2 * 16
+    slices = 16 * 2 * 256 * 128 * 2
+    bf16 = (4 + 256) * 16 * 2 * 128 * 2
+    qo = 16 * 128 * (2 + 4) + 16 * 4
+    assert got == idx + slices + bf16 + qo
+
+
 def test_decode_bytes_batch_counts_slices_once():
     w = synth.WORKLOADS["ouro14_g32_b32"]
     one = bench.decode_bytes_per_launch(w, _Lay(16), [1000], [128])
