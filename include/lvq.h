@@ -20,11 +20,16 @@
  *   - attention at loop step t reads only the step-t slice of each codebook,
  *     applies RoPE to the reconstructed keys, splits the coded tokens
  *     Flash-Decoding style and merges the splits with the bf16 tokens by
- *     logsumexp.
+ *     logsumexp;
+ *   - codebooks come from k-means over joint vectors (here the plain,
+ *     unweighted form: lvq_encode_prefill assigns, lvq_kmeans_update moves
+ *     the entries).
  *
  * Conventions for every entry point:
  *   - The caller owns every buffer (device memory unless stated).  The
- *     library allocates nothing and keeps no global state.
+ *     library allocates nothing and keeps no global state, apart from the
+ *     fixed workspace of lvq_decode_attention_noalloc and the settings of the
+ *     lvq_debug_faults test hook.
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
  *     NULL is the legacy default stream).  Errors the host can see (bad
  *     config, null or misaligned pointer, out-of-range argument) return at
