@@ -285,7 +285,10 @@ LVQ_API lvq_status lvq_dequantize(const lvq_config* cfg, const lvq_layout* lay, 
  *   - the call allocates nothing (no cudaMalloc or allocating library
  *     routine); it zeroes the merge counters with cudaMemsetAsync on `stream`;
  *   - the first call on a device looks up the array's device address with that
- *     device current; make that first call before any stream capture;
+ *     device current (cudaGetSymbolAddress), and looks it up again only when the
+ *     device's current context has changed (e.g. after cudaDeviceReset); make
+ *     that first call before any stream capture.  The lookup is guarded by a
+ *     lock, so concurrent first calls from several host threads are safe;
  *   - every call shares the one array: calls that overlap on the GPU (other
  *     streams, other host threads, other decode calls in flight) race and must
  *     be serialized by the caller. */

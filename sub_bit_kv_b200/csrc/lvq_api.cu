@@ -2,6 +2,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "lvq_common.cuh"
 
 using namespace lvq;
@@ -285,16 +287,40 @@ namespace {
 constexpr size_t kNoallocWorkspaceBytes = size_t(4) << 20;   // the stated maximum: 4 MiB
 static __device__ __align__(256) float g_noalloc_workspace[kNoallocWorkspaceBytes / sizeof(float)];
 
-// Device address of g_noalloc_workspace, looked up once per device with that
-// device current.  In host code the array's name is only a stand-in, never a
-// device address.
+// Device address of g_noalloc_workspace for the current device and context.  In host code
+// the array's name is only a stand-in, never a device address, so the address is looked up
+// with cudaGetSymbolAddress with that device current: once per device, and again only if the
+// device's current context changed since (after cudaDeviceReset the module is loaded anew and
+// the array may move).  The lookup runs under a lock, so host threads that make their first
+// calls at the same time do not race on the cache.
+using PFN_ctx_get_current = CUresult (*)(CUcontext*);
+
+CUcontext current_context() {
+  static PFN_ctx_get_current fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_ctx_get_current>(p);
+  }();
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
 float* noalloc_workspace(int dev) {
+  static std::mutex mu;
+  static CUcontext ctx[kMaxDevices] = {};
   static float* addr[kMaxDevices] = {};
   if (dev < 0 || dev >= kMaxDevices) return nullptr;
-  if (!addr[dev]) {
+  const CUcontext cur = current_context();
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev] || ctx[dev] != cur) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_workspace) != cudaSuccess) return nullptr;
     addr[dev] = static_cast<float*>(p);
+    ctx[dev] = cur;
   }
   return addr[dev];
 }

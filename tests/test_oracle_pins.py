@@ -47,6 +47,33 @@ def test_entries_reencode_to_own_index_and_duplicates_go_low():
     assert O.near_tie(d1b, d2b).all()
 
 
+def test_near_tie_fixture():
+    """The near-tie rule that decides which GPU/oracle code mismatches are acceptable:
+    relative to d1, inclusive at the bound, and only exact duplicates when d1 = 0."""
+    fx = _golden("near_tie.json")
+    d1 = np.array([c["d1"] for c in fx["cases"]])
+    d2 = np.array([c["d2"] for c in fx["cases"]])
+    assert O.NEAR_TIE_REL == fx["rel"]
+    got = O.near_tie(d1, d2)
+    assert got.tolist() == [c["tie"] for c in fx["cases"]], [c["why"] for c, g in zip(fx["cases"], got)
+                                                             if g != c["tie"]]
+
+
+def test_near_tie_from_nearest_entry_geometry():
+    """Distances from nearest_entry feed near_tie: x exactly between two entries is a tie;
+    moved off the midpoint by a hand-chosen amount it is or is not, as the relative gap says."""
+    C = np.zeros((256, 2))
+    C[:, 0] = 1000.0                     # every other entry far away
+    C[3] = [0.0, 0.0]
+    C[9] = [2.0, 0.0]
+    for shift, tie in ((0.0, True), (2.0 ** -22, True), (2.0 ** -18, False)):
+        x = np.array([[1.0 - shift, 0.0]])   # d1 = (1 - shift)^2, d2 = (1 + shift)^2
+        idx, d1, d2 = O.nearest_entry(x, C)
+        assert idx[0] == 3
+        # gap 4 * shift over d1 ~ 1: 2^-20 = 9.5e-7 <= 1e-6 (tie), 2^-16 = 1.5e-5 (not)
+        assert bool(O.near_tie(d1, d2)[0]) == tie
+
+
 def test_tc1_encode_matches_cdist_argmin():
     """At Tc = 1 the joint vector is G channels of one step: textbook VQ."""
     rng = np.random.default_rng(5)
@@ -458,6 +485,16 @@ def test_pins_catch_planted_mistakes(monkeypatch):
     with pytest.raises(AssertionError):
         test_kmeans_empty_entry_keeps_its_value()
     monkeypatch.undo()
+
+    # near-tie rule: a looser bound, an absolute gap, a strict inequality, relative to d2
+    for mutant in (lambda d1, d2: (d2 - d1) <= 1e-3 * d1,
+                   lambda d1, d2: (d2 - d1) <= 1e-6,
+                   lambda d1, d2: (d2 - d1) < 1e-6 * d1,
+                   lambda d1, d2: (d2 - d1) <= 1e-6 * d2):
+        monkeypatch.setattr(O, "near_tie", mutant)
+        with pytest.raises(AssertionError):
+            test_near_tie_fixture()
+        monkeypatch.undo()
 
     def round_via_fp32(x):                      # double rounding fp64 -> fp32 -> bf16
         return torch.tensor(np.asarray(x, dtype=np.float32)).to(torch.bfloat16).to(torch.float64).numpy()

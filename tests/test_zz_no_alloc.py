@@ -9,13 +9,19 @@ give what lvq_decode_attention gives with a caller-owned workspace.
 """
 import dataclasses
 
+import numpy as np
 import pytest
 import torch
 
-from sub_bit_kv_b200 import lvq, synth
+from sub_bit_kv_b200 import _build, lvq, synth
 from tests import _helpers as Hl
 
 pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _library():
+    _build.build()
 
 
 def _call(case, fn, layer, step, q, ns, **extra):
@@ -31,8 +37,6 @@ def _call(case, fn, layer, step, q, ns, **extra):
 
 
 def test_noalloc_decode_matches_workspace_decode_twice():
-    from sub_bit_kv_b200 import _build
-    _build.build()
     w = dataclasses.replace(synth.WORKLOADS["ouro14_g16_32k"], n_layers=2, n_kv_heads=2, n_q_heads=2)
     case = Hl.build_case(w, layers=2, ctx=[1900, 700], max_splits=16)
     assert case.cache.lay.workspace_bytes <= 4 << 20
@@ -43,9 +47,34 @@ def test_noalloc_decode_matches_workspace_decode_twice():
         out, lse = _call(case, lvq.lvq_decode_attention_noalloc, layer, step, q, ns)
         assert float((out - ref_out).abs().max()) <= Hl.OUT_ATOL
         assert float((lse - ref_lse).abs().max()) <= Hl.LSE_REL * max(1.0, float(ref_lse.abs().max()))
+        # and directly against the fp64 oracle, every request and head
+        for b in range(2):
+            for hq in range(w.n_q_heads):
+                ro, rl, _ = Hl.oracle_decode(case, layer, step, b, hq, q.cpu())
+                assert float(np.abs(out[b, hq].numpy() - ro).max()) <= Hl.OUT_ATOL
+                Hl.assert_lse_close(float(lse[b, hq]), rl, (b, hq))
+
+
+def test_noalloc_clears_the_counters_of_each_layout():
+    """The merge counters sit after the partials, so their place in the shared array moves
+    with the layout.  A call with many splits fills the array's start with partials; a
+    following call whose layout puts its counters inside that region must clear them
+    before its kernel runs (else the last CTA of a head is never recognised)."""
+    w = dataclasses.replace(synth.WORKLOADS["ouro14_g16_32k"], n_layers=1, n_kv_heads=4, n_q_heads=4)
+    big = Hl.build_case(w, layers=1, ctx=[3000], max_splits=96)
+    small = Hl.build_case(w, layers=1, ctx=[2500], max_splits=4)
+    # the small layout's counters lie inside the big layout's partial region
+    assert small.cache.lay.workspace_bytes < big.cache.lay.workspace_bytes <= 4 << 20
+    for rnd in range(2):
+        q = synth.queries(w, 0, 2, batch=1, token=rnd).cuda()
+        _call(big, lvq.lvq_decode_attention_noalloc, 0, 2, q, 96)
+        out, lse = _call(small, lvq.lvq_decode_attention_noalloc, 0, 2, q, 3)
+        ref_out, ref_lse = _call(small, lvq.lvq_decode_attention, 0, 2, q, 3, ws=(small.cache.workspace,))
+        assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
 
 
 def test_noalloc_rejects_a_layout_beyond_its_array():
+    """Checked on the host before anything is launched."""
     w = dataclasses.replace(synth.WORKLOADS["ouro14_g16_32k"], n_layers=1)
     cfg = Hl.make_cfg(w, max_batch=64, max_ctx=1024, max_splits=256)
     lay = lvq.lvq_cache_layout(cfg)
