@@ -215,8 +215,15 @@ def test_split_count_sweep_agrees():
     case = Hl.build_case(w, layers=1, ctx=[4000])
     q = synth.queries(w, 0, 2).cuda()
     outs = [Hl.run_decode(case, 0, 2, q, ns)[0] for ns in (1, 2, 7, 16, 33, 64)]
+    # Every output is a convex combination of value elements, computed per split count in
+    # another fp32 order: a split's contraction sums 256 histogram-weighted entries (worst
+    # case 256 * 2^-24 of max|V|), its fixed-point weights are exact to n * 2^-31 of their sum,
+    # and the merge adds at most 2 * 64 + 1 weighted partials.  So any two split counts agree
+    # to (256 + 129 + 2) * 2^-24 + 4000 * 2^-31 < 2^-15 of the largest value magnitude.
+    vmax = max(float(case.cb[0][1].abs().max()), float(case.sink_kv[(0, 0)][1].abs().max()),
+               float(case.ring_kv[(0, 0)][1].abs().max()))
     for o in outs[1:]:
-        assert float((o - outs[0]).abs().max()) <= 1e-5
+        assert float((o - outs[0]).abs().max()) <= 2.0 ** -15 * vmax
 
 
 def test_step_slice_isolation_on_gpu():
@@ -239,9 +246,9 @@ def test_step_slice_isolation_on_gpu():
         poisoned = Hl.run_decode(case, 0, step, q, 8)
         c.cbp.copy_(saved)
         assert torch.isfinite(poisoned[0]).all()
-        # shared-memory histogram sums may add in another order: compare to fp32 rounding
-        assert float((clean[0] - poisoned[0]).abs().max()) <= 1e-5
-        assert float((clean[1] - poisoned[1]).abs().max()) <= 1e-5
+        # same inputs in the same order (the weight histogram is integer): bit-identical
+        assert torch.equal(clean[0], poisoned[0]) and torch.equal(clean[1], poisoned[1])
+        assert torch.equal(clean[2], poisoned[2])
 
 
 def test_identical_codes_zero_key_share_uniform_attention():
