@@ -80,6 +80,20 @@ __device__ inline bool mbar_wait(uint32_t bar, uint32_t parity, long max_iter) {
   return false;
 }
 
+// The same, for waits that may be long: each poll lets the thread sleep up to ~0.25 us
+// (woken early when the phase completes), so a waiting warp takes few issue slots.
+__device__ inline bool mbar_wait_sleep(uint32_t bar, uint32_t parity, long max_iter) {
+  for (long i = 0; i < max_iter; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok) : "r"(bar), "r"(parity), "r"(256) : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+
 __device__ inline void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
 }

@@ -20,32 +20,48 @@
 // direct form sum_j (X_j - C_kj)^2 -- exact for bf16 inputs -- lowest index on
 // ties.  So every code equals the fp64 brute-force answer.
 //
-// CTA: 512 threads, one per SM (it allocates all 512 TMEM columns).  Work items
-// are (K/V, block, head, 16-channel span) x 1024-token ranges.  The raw input
-// tile [Tc][128 tokens][16 channels] arrives by TMA (no multicast) into a
-// 2-stage ring; the 16 channels hold 16/c groups.  Two sets of 8 warps each own
-// 256 TMEM columns and alternate over the groups: build the group's A tile,
-// issue its UMMA, and run the argmin epilogue, so one set's epilogue overlaps
-// the other set's MMA.  In a set, warps w and w + 4 read the same TMEM lane
-// quadrant (32 rows) and split the 256 entries into halves.
+// One persistent CTA per SM (it allocates all 512 TMEM columns), warp-specialised:
+//  * warp 9 (one lane) streams raw input tiles [Tc][128 tokens][16 channels] by
+//    TMA (no multicast) into a 3-stage ring (full/empty mbarriers);
+//  * warp 8 (one lane) issues the UMMAs: group-tile k of an item goes to
+//    accumulator k % 2 (256 TMEM columns each) once its A tile is ready and the
+//    accumulator's previous contents have been read, and commits to that
+//    accumulator's "full" barrier;
+//  * warps 0-3 (team 0) and 4-7 (team 1) each own one accumulator and take every
+//    other group-tile; thread r of a team owns row r (TMEM lane r, one token).
+//    For the team's next group-tile it builds row r of the A tile from the raw
+//    tile (and the row's ||x||^2), then drains the current accumulator: all 256
+//    columns of its row in four 64-column loads, the accumulator released to the
+//    MMA warp as soon as the last load has landed.  Per 32-column block it keeps
+//    the block minimum (3-input min) and the block's columns within eps of it as
+//    a bit mask, made on the FMA pipe: with 2^k scaled so that any fp32 value
+//    below the threshold t gives (t - v) 2^k >= 1, a saturating FMA turns each
+//    column into an exact 0 or 1 and a packed FMA shifts them into two float
+//    accumulators (even and odd columns).  The row's code follows from its eight
+//    block minima and masks, with fp64 rescoring of near-ties.
+// Work items are (K/V, block, head, 16-channel span) x 8192-token ranges; the
+// item's B tiles (its 16/c codebooks) are rebuilt between items.
 #include "lvq_common.cuh"
 
 namespace lvq {
 
 namespace tc {
 
-constexpr int kThreads = 512;
-constexpr int kSetThreads = 256;    // one MMA set: 8 warps
-constexpr int kRows = 128;          // UMMA M
+constexpr int kTeamWarps = 4;                    // one accumulator per team, one row per thread
+constexpr int kMmaWarp = 2 * kTeamWarps;         // warp 8: UMMA issue
+constexpr int kTmaWarp = kMmaWarp + 1;           // warp 9: raw-tile TMA
+constexpr int kThreads = 32 * (kTmaWarp + 1);    // 320
+constexpr int kRows = 128;                       // UMMA M
 constexpr int kTileTokens = 128;
-constexpr int kItemTokens = 1024;   // tokens per work item (8 tiles)
-constexpr int kSpan = 16;           // channels per item (TMA box x: 32 bytes)
-constexpr int kRawStages = 2;
+constexpr int kItemTokens = 8192;                // tokens per work item (64 tiles)
+constexpr int kSpan = 16;                        // channels per item (TMA box x: 32 bytes)
+constexpr int kRawStages = 3;
+constexpr int kBlocks = kEntries / 32;           // 32-column blocks of a row
 
 template <int G, int C>
 struct Enc {
   static constexpr int TC = G / C;            // steps per block
-  static constexpr int NGC = kSpan / C;       // groups per item
+  static constexpr int NGC = kSpan / C;       // groups per item (even: the teams alternate)
   static constexpr int KP = G + 16;           // padded K: G elements, 3 bias columns, zeros
   static constexpr int KSTEPS = KP / 16;
   static constexpr int SBO = KP * 16;         // bytes between 8-row core-matrix groups
@@ -53,18 +69,16 @@ struct Enc {
   static constexpr int B_TILE = kEntries * KP * 2;
   static constexpr int RAW = TC * kTileTokens * kSpan * 2;
   static constexpr int OFF_B = 0;
-  static constexpr int OFF_A = OFF_B + NGC * B_TILE;
-  static constexpr int OFF_RAW = OFF_A + 2 * NGC * A_TILE;   // A slots: [tile parity][group]
+  static constexpr int OFF_A = OFF_B + NGC * B_TILE;                // [team][slot]
+  static constexpr int OFF_RAW = OFF_A + 4 * A_TILE;
   static constexpr int OFF_NMAX = OFF_RAW + kRawStages * RAW;
-  static constexpr int OFF_BAR = OFF_NMAX + 16 * 4;
-  static constexpr int OFF_BMIN = OFF_BAR + 8 * (kRawStages + 2);     // [2 sets][8 blocks][128 rows]
-  static constexpr int OFF_MASK = OFF_BMIN + 2 * (kEntries / 32) * kRows * 4;   // [2 sets][8 blocks][128 rows]
-  static constexpr int OFF_TMEM = OFF_MASK + 2 * (kEntries / 32) * kRows * 4;
-  // + alignment slack; at least 120 KB so that one CTA (holding all of TMEM) fits per SM
-  static constexpr int SMEM = (OFF_TMEM + 16 + 1024) > 120 * 1024 ? (OFF_TMEM + 16 + 1024) : 120 * 1024;
-  static_assert(NGC == 2 || NGC == 4, "two MMA sets alternate over the item's groups");
+  static constexpr int OFF_BAR = OFF_NMAX + 64;
+  static constexpr int NBAR = 2 * kRawStages + 4 + 2 + 2;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;                 // + alignment slack
+  static_assert(NGC == 2 || NGC == 4, "two teams alternate over the item's groups");
   static_assert(SMEM <= 227 * 1024, "shared memory of one CTA");
-  static_assert(KP % 16 == 0, "K steps");
+  static_assert(KP % 16 == 0 && G % 8 == 0, "K steps, 16-byte chunks of a row");
 };
 
 // K-major, no-swizzle UMMA shared-memory descriptor: core matrices of 8 rows x
@@ -95,7 +109,9 @@ __device__ inline uint32_t raw_off(int s, int r, int ch) {
 __device__ inline void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ inline void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ inline void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ inline void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(n) : "memory"); }
+__device__ inline void mbar_arrive1(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
+}
 
 __device__ inline void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
@@ -134,6 +150,95 @@ __device__ inline float fmin3(float a, float b, float c) {
   return d;
 }
 
+__device__ inline float fma_sat(float a, float b, float c) {
+  float d;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Candidate masks use a permuted bit order: column 2p of a block is bit 31 - p,
+// column 2p + 1 is bit 15 - p.  Column of mask bit b:
+__device__ inline int mask_col(int b) { return b >= 16 ? 2 * (31 - b) : 2 * (15 - b) + 1; }
+
+// Four 32-column blocks of a row (columns 0-31 and 32-63 of `ra`, then of `rb`), processed
+// in lockstep so that their chains overlap: each block's minimum bm[b], and its columns
+// v < bm[b] + eps as a bit mask in the permuted order above.  eps > 0 is at least
+// 2^-15 |bm| (so bm + eps > bm).
+__device__ inline void quad_min_mask(const uint32_t (&ra)[64], const uint32_t (&rb)[64], float eps, float (&bm)[4],
+                                     uint32_t (&mask)[4]) {
+  // column i of block b (both compile-time after unrolling: the arrays stay in registers)
+  auto V = [&](int b, int i) -> float { return __uint_as_float(b < 2 ? ra[32 * b + i] : rb[32 * (b - 2) + i]); };
+  float m[4][4];
+#pragma unroll
+  for (int b = 0; b < 4; ++b)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) m[b][u] = V(b, u);
+#pragma unroll
+  for (int i = 4; i < 28; i += 8)        // columns 4..27: four chains per block, two columns a step
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        m[b][u] = fmin3(m[b][u], V(b, i + 2 * u), V(b, i + 2 * u + 1));
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {          // columns 28..31
+    const float a0 = fmin3(m[b][0], V(b, 28), V(b, 29));
+    const float a1 = fmin3(m[b][1], V(b, 30), V(b, 31));
+    bm[b] = fminf(fmin3(a0, a1, m[b][2]), m[b][3]);
+  }
+  // Any fp32 v < tb lies at least 2^(e-24) below it (e the exponent of tb), so with
+  // k = 24 - e, (tb - v) 2^k >= 1 and sat(fma(v, -2^k, tb 2^k)) is exactly 1; any v >= tb
+  // gives exactly 0 (an overflow to infinity keeps the sign, so it saturates the same way).
+  float tb[4], nsc[4], c[4];
+  bool fast = true;
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    tb[b] = bm[b] + eps;
+    const uint32_t E = (__float_as_uint(tb[b]) >> 23) & 0xffu;   // biased exponent of tb
+    fast = fast && E >= 24u;
+    const float sc = __uint_as_float((278u - (E < 24u ? 24u : E)) << 23);   // 2^k, k = 151 - E
+    nsc[b] = -sc;
+    c[b] = tb[b] * sc;                                         // exact: a power-of-two scale
+  }
+  if (fast) {
+    // per block two accumulators (pairs 0-7 and 8-15) of s = 0/1 shifted in: exact integers
+    float2 lo[4], hi[4];
+    const float2 two = make_float2(2.f, 2.f);
+#pragma unroll
+    for (int b = 0; b < 4; ++b) lo[b] = hi[b] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int p = 0; p < 8; ++p)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const float s0 = fma_sat(V(b, 2 * p), nsc[b], c[b]);
+        const float s1 = fma_sat(V(b, 2 * p + 1), nsc[b], c[b]);
+        const float s2 = fma_sat(V(b, 2 * p + 16), nsc[b], c[b]);
+        const float s3 = fma_sat(V(b, 2 * p + 17), nsc[b], c[b]);
+        lo[b] = __ffma2_rn(lo[b], two, make_float2(s0, s1));
+        hi[b] = __ffma2_rn(hi[b], two, make_float2(s2, s3));
+      }
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      // 16-bit integers (pair 0 on top), plus 2^23 so that they sit in the low mantissa bits
+      const float2 m2 = __ffma2_rn(lo[b], make_float2(256.f, 256.f), hi[b]);
+      const float2 w = __fadd2_rn(m2, make_float2(8388608.f, 8388608.f));
+      mask[b] = __byte_perm(__float_as_uint(w.y), __float_as_uint(w.x), 0x5410);
+    }
+  } else {
+    // some tb is zero, subnormal or tiny: compare the plain way (sign of tb - v per column)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      uint32_t sa = 0u, sb = 0u;
+#pragma unroll
+      for (int p = 0; p < 16; ++p) {
+        sa = (sa << 1) | (tb[b] - V(b, 2 * p) > 0.f ? 1u : 0u);
+        sb = (sb << 1) | (tb[b] - V(b, 2 * p + 1) > 0.f ? 1u : 0u);
+      }
+      mask[b] = (sa << 16) | sb;
+    }
+  }
+}
+
 template <int G, int C>
 __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
     const __grid_constant__ CUtensorMap tmap, Geo g, int layer, int req, int tok_begin, int n_tok,
@@ -148,17 +253,19 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
   unsigned char* At = smem + X::OFF_A;
   unsigned char* raw = smem + X::OFF_RAW;
   float* nmax_s = reinterpret_cast<float*>(smem + X::OFF_NMAX);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + X::OFF_BAR);  // [0..1] raw stages, [2..3] MMA sets
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + X::OFF_TMEM);
-  volatile int* fail_s = reinterpret_cast<volatile int*>(smem + X::OFF_TMEM + 4);   // per MMA set
-  float* bmin_s = reinterpret_cast<float*>(smem + X::OFF_BMIN);
-  uint32_t* mask_s = reinterpret_cast<uint32_t*>(smem + X::OFF_MASK);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + X::OFF_BAR);
+  // bars: [0, NR) raw full, [NR, 2NR) raw empty, then A ready [team][slot], acc full [team], acc empty [team]
+  uint64_t* raw_full = bars;
+  uint64_t* raw_empty = bars + kRawStages;
+  uint64_t* a_ready = bars + 2 * kRawStages;
+  uint64_t* acc_full = a_ready + 4;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + X::OFF_MISC);
+  volatile int* fail_s = reinterpret_cast<volatile int*>(smem + X::OFF_MISC + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int set = tid / kSetThreads;      // MMA set: warps 0-7 or 8-15
-  const int hf = (warp >> 2) & 1;         // half of the 256 entries this warp scans
-  const int row = 32 * (warp & 3) + lane; // TMEM lane = tile row = token of the tile
-  const bool set_leader = (tid % kSetThreads) == 0;
+  const int team = warp / kTeamWarps;     // 0, 1 (2 for the MMA and TMA warps)
+  const int row = tid & (kRows - 1);      // TMEM lane = tile row = token of the tile (team warps)
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" :: "r"(smem_addr(tmem_slot))
@@ -166,85 +273,45 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (tid == 0) {
-    for (int i = 0; i < kRawStages + 2; ++i) mbar_init(smem_addr(&bars[i]), 1);
+    for (int i = 0; i < kRawStages; ++i) {
+      mbar_init(smem_addr(&raw_full[i]), 1);
+      mbar_init(smem_addr(&raw_empty[i]), 2 * kTeamWarps);
+    }
+    for (int i = 0; i < 4; ++i) mbar_init(smem_addr(&a_ready[i]), kTeamWarps);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_addr(&acc_full[i]), 1);
+      mbar_init(smem_addr(&acc_empty[i]), kTeamWarps);
+    }
     fence_mbar_init();
-    fail_s[0] = 0;
-    fail_s[1] = 0;
+    *fail_s = 0;
   }
-  // zero the A tiles once: the columns past G + 3 stay zero
-  for (int i = tid; i < 2 * NGC * X::A_TILE / 16; i += kThreads)
-    reinterpret_cast<uint4*>(At)[i] = make_uint4(0, 0, 0, 0);
+  // A tiles: [x | 1 1 1 | 0...]; the columns from G on never change
+  for (int i = tid; i < 4 * X::A_TILE / 16; i += kThreads) {
+    const int a = i / (X::A_TILE / 16), rem = i % (X::A_TILE / 16);
+    const int r = rem / (X::KP / 8), k8 = rem % (X::KP / 8);
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (k8 * 8 == G) v = make_uint4(0x3f803f80u, 0x3f80u, 0u, 0u);   // bf16 1.0 in columns G .. G+2
+    *reinterpret_cast<uint4*>(At + a * X::A_TILE + kmaj_off(r, k8 * 8, SBO)) = v;
+  }
+  fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t tmem_set = tmem_base + (uint32_t)(set * 256);
-  const uint32_t lane_addr = ((uint32_t)(32 * (warp & 3))) << 16;
-  float* const bmin_set = bmin_s + set * (kEntries / 32) * kRows;     // [8 blocks][128 rows]
-  uint32_t* const mask_set = mask_s + set * (kEntries / 32) * kRows;  // [8 blocks][128 rows]
+  const long wit = g.wait_iters;
 
   const int n_spans = g.d / kSpan;
   const int n_sets = 2 * g.nblk * g.H * n_spans;
   const int n_ranges = (n_tok + kItemTokens - 1) / kItemTokens;
   const long n_items = (long)n_sets * n_ranges;
 
-  // A row of this thread's token for group gib from a raw tile: element s*c+e =
-  // raw[s][row][gib*c+e].  Both threads of a row read it (for ||x||^2); each writes half of
-  // its 16-byte chunks.  Returns ||x||^2 of the joint vector.
-  auto build_a = [&](const unsigned char* src_tile, int gib, unsigned char* at) -> float {
-    uint32_t xw[G / 2];                  // the row's G elements, two per word
-#pragma unroll
-    for (int s2 = 0; s2 < TC; ++s2) {
-      const unsigned char* src = src_tile + raw_off(s2, row, gib * C);
-      if constexpr (C == 4) {
-        const uint2 w = *reinterpret_cast<const uint2*>(src);
-        xw[s2 * 2] = w.x;
-        xw[s2 * 2 + 1] = w.y;
-      } else {
-        const uint4 w = *reinterpret_cast<const uint4*>(src);
-        xw[s2 * 4] = w.x;
-        xw[s2 * 4 + 1] = w.y;
-        xw[s2 * 4 + 2] = w.z;
-        xw[s2 * 4 + 3] = w.w;
-      }
-    }
-    float x2 = 0.f;
-#pragma unroll
-    for (int q = 0; q < G / 2; ++q) {
-      const float lo = bf16_lo(xw[q]), hi = bf16_hi(xw[q]);
-      x2 = fmaf(lo, lo, x2);
-      x2 = fmaf(hi, hi, x2);
-    }
-#pragma unroll
-    for (int k8 = 0; k8 < G / 8; ++k8)
-      if ((k8 >= G / 16) == (hf == 1))
-        *reinterpret_cast<uint4*>(at + kmaj_off(row, k8 * 8, SBO)) =
-            make_uint4(xw[k8 * 4], xw[k8 * 4 + 1], xw[k8 * 4 + 2], xw[k8 * 4 + 3]);
-    if (hf == 1) {
-      const uint32_t one = 0x3f80u;   // bf16 1.0
-      *reinterpret_cast<uint4*>(at + kmaj_off(row, G, SBO)) = make_uint4(one | (one << 16), one, 0u, 0u);
-    }
-    fence_proxy_async();             // the tile is read by the tensor core (async proxy)
-    return x2;
-  };
-  // the set's UMMA of group gib from A slot aslot into the set's TMEM columns (one thread)
-  auto issue_mma = [&](int aslot, int gib) {
-    const uint32_t a0 = smem_addr(At + aslot * X::A_TILE), b0 = smem_addr(Bt + gib * X::B_TILE);
-#pragma unroll
-    for (int ks = 0; ks < X::KSTEPS; ++ks)
-      mma_bf16(tmem_set, smem_desc(a0 + ks * 256, SBO), smem_desc(b0 + ks * 256, SBO), kIdesc, ks > 0);
-    mma_commit(smem_addr(&bars[kRawStages + set]));
-  };
-  bool issued = false;              // the set's next MMA was issued during the previous group
-  bool outstanding = false;         // an MMA of this set may still be running
-  float xx_next = 0.f;
+  long T_glob = 0;          // raw tiles of the items before this one (this CTA)
+  long J_glob = 0;          // group-tiles per team of the items before this one
+  // in-flight bookkeeping for a failed run: the last MMA issued per accumulator, tiles issued
+  long last_mma[2] = {-1, -1};
+  long tiles_issued = 0;
 
-  uint32_t raw_phase = 0;   // bit s: parity of raw stage s
-  uint32_t mma_phase = 0;
-  int tile_counter = 0;     // tiles processed by this CTA (drives the raw ring)
-  bool failed = false;
-
-  for (long item = blockIdx.x; item < n_items && !failed; item += gridDim.x) {
+  for (long item = blockIdx.x; item < n_items; item += gridDim.x) {
     int cs = (int)(item / n_ranges);
     const int range = (int)(item % n_ranges);
     const int span = cs % n_spans; cs /= n_spans;
@@ -254,24 +321,17 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
     const int t_first = tok_begin + range * kItemTokens;
     const int t_last = min(tok_begin + n_tok, t_first + kItemTokens);
     const int n_tiles = (t_last - t_first + kTileTokens - 1) / kTileTokens;
+    const int n_j = n_tiles * NGC / 2;              // group-tiles per team
     uint8_t* const idx_item = idx + idx_stream_off(g, layer, blk, req, h, kvi);
 
-    // all MMAs of the previous item have completed (each set waited for its commits)
+    // every role has finished the previous item: its MMAs completed (the teams waited for
+    // each), its raw tiles landed (the teams waited for each)
     __syncthreads();
-    // prefetch the first two raw tiles of this item
-    if (tid == 0) {
-      for (int tl = 0; tl < min(2, n_tiles); ++tl) {
-        const int stg = (tile_counter + tl) % kRawStages;
-        const uint32_t bar = smem_addr(&bars[stg]);
-        mbar_expect_tx(bar, X::RAW);
-        tma_load_3d(smem_addr(raw + stg * X::RAW), &tmap, h * g.d + span * kSpan, t_first + tl * kTileTokens,
-                    kvi * g.T + blk * TC, bar);
-      }
-    }
-    // B tiles: [-2 C_k | n1 n2 n3 | 0] for the item's groups, K-major no-swizzle;
-    // nmax_s[gi] = max_k ||C_k||^2 (non-negative floats order like their bits)
+    if (*fail_s) break;
     if (tid < NGC) nmax_s[tid] = 0.f;
     __syncthreads();
+    // B tiles: [-2 C_k | n1 n2 n3 | 0] for the item's groups, K-major no-swizzle;
+    // nmax_s[gi] = max_k ||C_k||^2 (non-negative floats order like their bits)
     for (int e = tid; e < NGC * kEntries; e += kThreads) {
       const int gi = e / kEntries, k = e % kEntries;
       const int grp = span * NGC + gi;
@@ -306,175 +366,219 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
     fence_proxy_async();
     __syncthreads();
 
-    for (int tl = 0; tl < n_tiles && !failed; ++tl, ++tile_counter) {
-      const int stg = tile_counter % kRawStages;
-      const int t0 = t_first + tl * kTileTokens;
-      if (__syncthreads_or(!mbar_wait(smem_addr(&bars[stg]), (raw_phase >> stg) & 1u, g.wait_iters))) {
-        failed = true;
-        break;
+    if (warp == kTmaWarp) {
+      // ---- raw tiles of the item, through the ring
+      if (lane == 0) {
+        for (int t = 0; t < n_tiles; ++t) {
+          const long T = T_glob + t;
+          const int stg = (int)(T % kRawStages);
+          if (T >= kRawStages &&
+              (*fail_s || !mbar_wait_sleep(smem_addr(&raw_empty[stg]), (uint32_t)((T / kRawStages - 1) & 1), wit))) {
+            *fail_s = 1;
+            break;
+          }
+          const uint32_t bar = smem_addr(&raw_full[stg]);
+          mbar_expect_tx(bar, X::RAW);
+          tma_load_3d(smem_addr(raw + stg * X::RAW), &tmap, h * g.d + span * kSpan, t_first + t * kTileTokens,
+                      kvi * g.T + blk * TC, bar);
+          tiles_issued = T + 1;
+        }
       }
-      raw_phase ^= 1u << stg;
-      const unsigned char* rw = raw + stg * X::RAW;
-      const bool valid_row = t0 + row < t_last;
-
-      // each set handles groups gi = set, set + 2, ...  The A tile of the set's next group is
-      // built while the current group's MMA runs (A slots alternate with the tile parity), and
-      // that next MMA is issued as soon as the current one's accumulator has been read.
-      for (int gi = set; gi < NGC; gi += 2) {
-        const int slot = gi + NGC * (tile_counter & 1);
-        float xx;
-        if (issued) {
-          xx = xx_next;
-          issued = false;
-        } else {
-          xx = build_a(rw, gi, At + slot * X::A_TILE);
-          tc_fence_before();
-          named_sync(1 + set, kSetThreads);
-          if (set_leader) issue_mma(slot, gi);
-          outstanding = true;
+    } else if (warp == kMmaWarp) {
+      // ---- UMMAs: group-tile k of the item goes to accumulator k % 2
+      if (lane == 0) {
+        for (int k = 0; k < n_tiles * NGC; ++k) {
+          const int tm = k & 1;
+          const long J = J_glob + (k >> 1);
+          const int slot = (int)(J & 1);
+          if (*fail_s || !mbar_wait_sleep(smem_addr(&a_ready[tm * 2 + slot]), (uint32_t)((J >> 1) & 1), wit) ||
+              (J >= 1 && !mbar_wait_sleep(smem_addr(&acc_empty[tm]), (uint32_t)((J - 1) & 1), wit))) {
+            *fail_s = 1;
+            break;
+          }
+          tc_fence_after();
+          const int gi = k % NGC;
+          const uint32_t a0 = smem_addr(At + (tm * 2 + slot) * X::A_TILE), b0 = smem_addr(Bt + gi * X::B_TILE);
+#pragma unroll
+          for (int ks = 0; ks < X::KSTEPS; ++ks)
+            mma_bf16(tmem_base + (uint32_t)(tm * 256), smem_desc(a0 + ks * 256, SBO), smem_desc(b0 + ks * 256, SBO),
+                     kIdesc, ks > 0);
+          mma_commit(smem_addr(&acc_full[tm]));
+          last_mma[tm] = J;
         }
-        int next_slot = -1, next_gi = 0;
-        if (gi + 2 < NGC) {
-          next_slot = slot + 2;
-          next_gi = gi + 2;
-          xx_next = build_a(rw, next_gi, At + next_slot * X::A_TILE);
-        } else if (tl + 1 < n_tiles) {
-          // the set's first group of the next tile: its raw stage was requested two tiles ago
-          const int stg1 = (tile_counter + 1) % kRawStages;
-          if (mbar_wait(smem_addr(&bars[stg1]), (raw_phase >> stg1) & 1u, g.wait_iters)) {
-            next_slot = set + NGC * ((tile_counter + 1) & 1);
-            next_gi = set;
-            xx_next = build_a(raw + stg1 * X::RAW, set, At + next_slot * X::A_TILE);
+      }
+    } else {
+      // ---- a team: group-tiles j = 0, 1, ... of the item are k = 2 j + team
+      const uint32_t tmem_acc = tmem_base + (uint32_t)(team * 256) + ((uint32_t)(32 * (warp & 3)) << 16);
+      // builds row `row` of the A tile of team group-tile j; returns ||x||^2 of the row, or a
+      // negative value if a wait timed out (uniform over the warp)
+      auto build = [&](int j) -> float {
+        const int k = 2 * j + team, t = k / NGC, gi = k % NGC;
+        const long T = T_glob + t, J = J_glob + j;
+        const int stg = (int)(T % kRawStages);
+        const bool ok = !*fail_s && mbar_wait_sleep(smem_addr(&raw_full[stg]), (uint32_t)((T / kRawStages) & 1), wit);
+        if (__any_sync(0xffffffffu, !ok)) return -1.f;
+        const unsigned char* rw = raw + stg * X::RAW;
+        unsigned char* at = At + (team * 2 + (int)(J & 1)) * X::A_TILE;
+        uint32_t xw[G / 2];
+#pragma unroll
+        for (int s2 = 0; s2 < TC; ++s2) {
+          const unsigned char* src = rw + raw_off(s2, row, gi * C);
+          if constexpr (C == 4) {
+            const uint2 w = *reinterpret_cast<const uint2*>(src);
+            xw[s2 * 2] = w.x;
+            xw[s2 * 2 + 1] = w.y;
           } else {
-            fail_s[set] = 1;
+            const uint4 w = *reinterpret_cast<const uint4*>(src);
+            xw[s2 * 4] = w.x;
+            xw[s2 * 4 + 1] = w.y;
+            xw[s2 * 4 + 2] = w.z;
+            xw[s2 * 4 + 3] = w.w;
           }
         }
-        // one warp of the set waits for the MMA; the barrier releases the others (no spinning)
-        if ((tid % kSetThreads) < 32) {
-          __syncwarp();
-          if (!mbar_wait(smem_addr(&bars[kRawStages + set]), mma_phase, g.wait_iters)) fail_s[set] = 1;
+        float2 x2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < G / 2; ++q) {
+          const float2 v = make_float2(bf16_lo(xw[q]), bf16_hi(xw[q]));
+          x2 = __ffma2_rn(v, v, x2);
         }
-        named_sync(1 + set, kSetThreads);
+#pragma unroll
+        for (int c8 = 0; c8 < G / 8; ++c8)
+          *reinterpret_cast<uint4*>(at + kmaj_off(row, c8 * 8, SBO)) =
+              make_uint4(xw[c8 * 4], xw[c8 * 4 + 1], xw[c8 * 4 + 2], xw[c8 * 4 + 3]);
+        fence_proxy_async();             // the tile is read by the tensor core (async proxy)
+        __syncwarp();
+        if (lane == 0) mbar_arrive1(smem_addr(&a_ready[team * 2 + (int)(J & 1)]));
+        return x2.x + x2.y;
+      };
+      float xx_cur = n_j > 0 ? build(0) : 0.f;
+      bool ok = xx_cur >= 0.f;
+      for (int j = 0; j < n_j && ok; ++j) {
+        const int k = 2 * j + team, t = k / NGC, gi = k % NGC;
+        const long J = J_glob + j, T = T_glob + t;
+        const int stg = (int)(T % kRawStages);
+        float xx_next = 0.f;
+        if (j + 1 < n_j) {
+          xx_next = build(j + 1);
+          ok = xx_next >= 0.f;
+        }
+        if (ok) ok = !*fail_s && mbar_wait_sleep(smem_addr(&acc_full[team]), (uint32_t)(J & 1), wit);
+        if (__any_sync(0xffffffffu, !ok)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-
-        // epilogue, one pass over this warp's half of the row (four 32-column blocks, two
-        // 64-column loads): each block's minimum, and the block's columns within eps of that
-        // minimum as a bit mask (bit 31 - i for column i).  Of the block holding the row
-        // minimum, that mask is exactly the row's candidates inside it; of any other block it
-        // holds every candidate of the row in that block (its minimum is not below the row's).
-        const float eps = (xx + nmax_s[gi]) * 0x1p-14f;
-#pragma unroll 1
-        for (int q2 = 0; q2 < 2; ++q2) {
-          uint32_t ra[64];
-          tmem_ld64_nowait(tmem_set + lane_addr + hf * 128 + q2 * 64, ra);
+        // eps = 2^-14 (||x||^2 + max ||C||^2), at least 2^-120 so that bm + eps > bm always
+        const float eps = fmaxf((xx_cur + nmax_s[gi]) * 0x1p-14f, 0x1p-120f);
+        float bmin[kBlocks];
+        uint32_t mask[kBlocks];
+        {
+          uint32_t ra[64], rb[64];
+          tmem_ld64_nowait(tmem_acc + 0, ra);
+          tmem_ld64_nowait(tmem_acc + 64, rb);
           tmem_wait_ld();
+          float q0[4], q1[4];
+          uint32_t k0[4], k1[4];
+          quad_min_mask(ra, rb, eps, q0, k0);
+          tmem_ld64_nowait(tmem_acc + 128, ra);
+          tmem_ld64_nowait(tmem_acc + 192, rb);
+          tmem_wait_ld();
+          // every column of the row is in registers: the accumulator may be overwritten
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive1(smem_addr(&acc_empty[team]));
+          quad_min_mask(ra, rb, eps, q1, k1);
 #pragma unroll
-          for (int b2 = 0; b2 < 2; ++b2) {
-            const uint32_t* r = ra + 32 * b2;
-            float m0 = __uint_as_float(r[0]), m1 = __uint_as_float(r[1]);
-#pragma unroll
-            for (int i = 2; i < 30; i += 4) {          // columns 2..29
-              m0 = fmin3(m0, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
-              m1 = fmin3(m1, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
-            }
-            m0 = fmin3(m0, __uint_as_float(r[30]), __uint_as_float(r[31]));
-            const float bm = fminf(m0, m1);
-            // sign of (bm + eps) - v per column, shifted in: 1 = outside the window
-            const float tb = bm + eps;
-            const float2 t2 = make_float2(tb, tb), neg1 = make_float2(-1.f, -1.f);
-            uint32_t sg = 0u;
-#pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-              const float2 e = __ffma2_rn(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), neg1, t2);
-              sg = __funnelshift_l(__float_as_uint(e.x), sg, 1);
-              sg = __funnelshift_l(__float_as_uint(e.y), sg, 1);
-            }
-            const int q = hf * 4 + q2 * 2 + b2;
-            bmin_set[q * kRows + row] = bm;
-            mask_set[q * kRows + row] = ~sg;
+          for (int b = 0; b < 4; ++b) {
+            bmin[b] = q0[b];
+            bmin[4 + b] = q1[b];
+            mask[b] = k0[b];
+            mask[4 + b] = k1[b];
           }
         }
-        tc_fence_before();
-        named_sync(1 + set, kSetThreads);      // also: every thread saw the MMA wait's outcome
-        const bool ok = fail_s[set] == 0;      // uniform over the set
-        if (ok) outstanding = false;
-        mma_phase ^= 1u;                       // one completed phase of this set's barrier per group
-        // the accumulator has been read: start the next group's MMA (its A tile was completed by
-        // every thread of the set before the barrier above)
-        if (ok && next_slot >= 0) {
-          if (set_leader) {
-            tc_fence_after();
-            issue_mma(next_slot, next_gi);
-          }
-          issued = true;
-          outstanding = true;
-        }
-        float bmin[kEntries / 32];
-#pragma unroll
-        for (int q = 0; q < kEntries / 32; ++q) bmin[q] = bmin_set[q * kRows + row];
-        float mrow = bmin[0];
-#pragma unroll
-        for (int q = 1; q < kEntries / 32; ++q) mrow = fminf(mrow, bmin[q]);
+        const float mrow = fminf(fmin3(bmin[0], bmin[1], bmin[2]), fmin3(bmin[3], bmin[4], fmin3(bmin[5], bmin[6], bmin[7])));
         const float thr = mrow + eps;
         uint32_t bmask = 0, at_min = 0;   // blocks that can hold a candidate / that hold the minimum
 #pragma unroll
-        for (int q = 0; q < kEntries / 32; ++q) {
-          bmask |= (bmin[q] <= thr ? 1u : 0u) << q;
-          at_min |= (bmin[q] == mrow ? 1u : 0u) << q;
+        for (int q = 0; q < kBlocks; ++q) {
+          bmask |= bmin[q] <= thr ? 1u << q : 0u;
+          at_min |= bmin[q] == mrow ? 1u << q : 0u;
         }
-        const int wb = at_min ? __ffs(at_min) - 1 : 0;   // the first block holding the minimum
-        const bool mine = (wb >> 2) == hf;     // this thread's half holds it: it owns the row
-        const uint32_t cm = mask_set[wb * kRows + row];
-        int code = wb * 32 + __clz(cm);
-        const bool tie = mine && valid_row && (__popc(cm) + __popc(bmask & ~(1u << wb)) > 1);
-        if (tie) {
-          // near-tie: exact fp64 direct-form distances of the candidates of every block within
-          // eps (the block masks are supersets of them), lowest index on ties
-          const unsigned char* bt = Bt + gi * X::B_TILE;
-          double best = 1e300;
-          int bk = kEntries;
-          for (uint32_t wm = bmask; wm; wm &= wm - 1u) {
-            const int q = __ffs(wm) - 1;
-            for (uint32_t m = mask_set[q * kRows + row]; m; m &= m - 1u) {
-              const int k = q * 32 + 32 - __ffs(m);       // bit 31 - i holds column i
-              double d2 = 0.0;                           // sum_j (x_j - C_kj)^2; the tile holds -2 C
+        const int wb = __ffs(at_min) - 1;               // the first block holding the minimum
+        // mask[wb] by a three-level select on the bits of wb
+        const uint32_t c01 = wb & 1 ? mask[1] : mask[0], c23 = wb & 1 ? mask[3] : mask[2];
+        const uint32_t c45 = wb & 1 ? mask[5] : mask[4], c67 = wb & 1 ? mask[7] : mask[6];
+        const uint32_t c03 = wb & 2 ? c23 : c01, c47 = wb & 2 ? c67 : c45;
+        const uint32_t cm = wb & 4 ? c47 : c03;
+        const int t0 = t_first + t * kTileTokens;
+        if (t0 + row < t_last) {
+          int code = wb * 32 + mask_col(31 - __clz(cm));
+          if (__popc(cm) + __popc(bmask & ~(1u << wb)) > 1) {
+            // near-tie: exact fp64 direct-form distances of the candidates of every block within
+            // eps (the block masks are supersets of them), lowest index on ties
+            const unsigned char* bt = Bt + gi * X::B_TILE;
+            const unsigned char* rw = raw + stg * X::RAW;
+            float xf[G];                                    // the row's joint vector, element s*c + e
 #pragma unroll
-              for (int s2 = 0; s2 < TC; ++s2)
+            for (int s2 = 0; s2 < TC; ++s2)
 #pragma unroll
-                for (int e = 0; e < C; ++e) {
-                  const int j = s2 * C + e;
-                  const uint32_t cw = *reinterpret_cast<const uint32_t*>(bt + kmaj_off(k, j & ~1, SBO));
-                  const float c2 = (j & 1) ? bf16_hi(cw) : bf16_lo(cw);
-                  const float xf = __bfloat162float(
-                      *reinterpret_cast<const __nv_bfloat16*>(rw + raw_off(s2, row, gi * C + e)));
-                  const double df = (double)xf + 0.5 * (double)c2;
-                  d2 = fma(df, df, d2);
+              for (int e = 0; e < C; ++e)
+                xf[s2 * C + e] = __bfloat162float(
+                    *reinterpret_cast<const __nv_bfloat16*>(rw + raw_off(s2, row, gi * C + e)));
+            double best = 1e300;
+            int bk = kEntries;
+#pragma unroll 1
+            for (int q = 0; q < kBlocks; ++q) {
+              if (!((bmask >> q) & 1u)) continue;
+              for (uint32_t m = mask[q]; m; m &= m - 1u) {
+                const int kk = q * 32 + mask_col(__ffs(m) - 1);
+                // sum_j (x_j - C_kj)^2 in two chains; the tile holds -2 C (exact halving)
+                double d2a = 0.0, d2b = 0.0;
+#pragma unroll
+                for (int j8 = 0; j8 < G / 8; ++j8) {
+                  const uint4 cw = *reinterpret_cast<const uint4*>(bt + kmaj_off(kk, j8 * 8, SBO));
+                  const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+                  for (int q2 = 0; q2 < 4; ++q2) {
+                    const double da = (double)xf[j8 * 8 + 2 * q2] + 0.5 * (double)bf16_lo(w4[q2]);
+                    const double db = (double)xf[j8 * 8 + 2 * q2 + 1] + 0.5 * (double)bf16_hi(w4[q2]);
+                    d2a = fma(da, da, d2a);
+                    d2b = fma(db, db, d2b);
+                  }
                 }
-              if (d2 < best || (d2 == best && k < bk)) { best = d2; bk = k; }
+                const double d2 = d2a + d2b;
+                if (d2 < best || (d2 == best && kk < bk)) { best = d2; bk = kk; }
+              }
             }
+            code = bk;
           }
-          code = bk;
-        }
-        if (mine && valid_row && ok) {
           const int cn = coded_offset + (t0 + row - tok_begin);
           idx_item[(size_t)(cn >> 3) * g.page_bytes + (span * NGC + gi) * kPage + (cn & 7)] = (uint8_t)code;
         }
-        if (!ok) break;
+        // the last group-tile of raw tile t for this team: the stage may be refilled
+        if (gi + 2 >= NGC) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive1(smem_addr(&raw_empty[stg]));
+        }
+        xx_cur = xx_next;
       }
-      fence_proxy_async();   // this thread's reads of the raw stage before its refill by TMA
-      if (__syncthreads_or(fail_s[0] | fail_s[1])) failed = true;
-      // refill this raw stage with the tile two ahead
-      if (tid == 0 && tl + 2 < n_tiles) {
-        const uint32_t bar = smem_addr(&bars[stg]);
-        mbar_expect_tx(bar, X::RAW);
-        tma_load_3d(smem_addr(raw + stg * X::RAW), &tmap, h * g.d + span * kSpan, t0 + 2 * kTileTokens,
-                    kvi * g.T + blk * TC, bar);
-      }
+      if (!ok && lane == 0) *fail_s = 1;
     }
+    T_glob += n_tiles;
+    J_glob += n_j;
   }
-  if (failed && tid == 0) set_status(st, LVQ_ETIMEOUT);
-  if (failed && set_leader && outstanding)   // let a set's last MMA finish before TMEM is freed
-    mbar_wait(smem_addr(&bars[kRawStages + set]), mma_phase, g.wait_iters);
+  __syncthreads();
+  const bool failed = *fail_s != 0;
+  if (failed) {
+    if (tid == 0) set_status(st, LVQ_ETIMEOUT);
+    // let every issued MMA and tile copy finish before TMEM and shared memory are released
+    if (warp == kMmaWarp && lane == 0)
+      for (int tm = 0; tm < 2; ++tm)
+        if (last_mma[tm] >= 0) mbar_wait(smem_addr(&acc_full[tm]), (uint32_t)(last_mma[tm] & 1), wit);
+    if (warp == kTmaWarp && lane == 0)
+      for (long T = tiles_issued - kRawStages; T < tiles_issued; ++T)
+        if (T >= 0) mbar_wait(smem_addr(&raw_full[T % kRawStages]), (uint32_t)((T / kRawStages) & 1), wit);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
