@@ -173,11 +173,15 @@ LVQ_API lvq_status lvq_rope_table(const lvq_config* cfg, const lvq_layout* lay, 
 /* Prefill encode ("LoopVQ summary", "premises and limits": the keys and values
  * of every loop step are kept until the last step, then each joint vector is
  * encoded against the codebook).
- *   layer: 0..n_layers-1; req: request 0..max_batch-1.
+ *   layer: 0..n_layers-1, or -1 for every layer in one call.
+ *   req: request 0..max_batch-1.
  *   kv: device bf16 [2][T][n_tok_total][Hkv][d] pre-RoPE keys (kv=0) and values
  *       (kv=1) of one layer and request; kv_tok_stride is the element stride
  *       between consecutive tokens (>= Hkv*d); the step stride is
- *       kv_tok_stride * kv_tokens and the K/V stride T times that.
+ *       kv_tok_stride * kv_tokens and the K/V stride T times that.  With
+ *       layer = -1 it holds every layer, [n_layers][2][T][...], the layer
+ *       stride 2 T times the step stride; the tensor-core encoder then spreads
+ *       all layers' work over one persistent launch.
  *   kv_tokens: tokens in kv (its token extent).
  *   tok_begin, n_tok: tokens [tok_begin, tok_begin + n_tok) of kv are encoded
  *       into coded slots [coded_offset, coded_offset + n_tok).

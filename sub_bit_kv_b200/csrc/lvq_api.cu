@@ -161,7 +161,7 @@ lvq_status lvq_encode_prefill(const lvq_config* cfg, const lvq_layout* lay, int3
   Geo g;
   lvq_status s = check_all(cfg, lay, &g);
   if (s != LVQ_OK) return s;
-  if (layer < 0 || layer >= g.L || req < 0 || req >= g.B || n_tok < 0 || tok_begin < 0 ||
+  if (layer < -1 || layer >= g.L || req < 0 || req >= g.B || n_tok < 0 || tok_begin < 0 ||
       kv_tokens < 0 || (int64_t)tok_begin + n_tok > kv_tokens || coded_offset < 0 ||
       (int64_t)coded_offset + n_tok > (int64_t)g.P * kPage || kv_tok_stride < (int64_t)g.H * g.d)
     return LVQ_EINVAL;

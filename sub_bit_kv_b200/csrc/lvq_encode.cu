@@ -84,6 +84,15 @@ cudaError_t launch_encode_prefill(const Geo& g, int layer, int req, const __nv_b
                                   int32_t* st, cudaStream_t s) {
   (void)st;
   if (n_tok == 0) return cudaSuccess;
+  if (layer < 0) {   // every layer: kv holds the layers back to back, one launch each
+    const int64_t layer_stride = (int64_t)2 * g.T * kv_tokens * tok_stride;
+    for (int l = 0; l < g.L; ++l) {
+      const cudaError_t e = launch_encode_prefill(g, l, req, kv + l * layer_stride, tok_stride, kv_tokens, tok_begin,
+                                                  n_tok, coded_offset, cb, idx, st, s);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
 #define LVQ_ENC(GG, CC)                                                                          \
   if (g.G == GG && g.c == CC)                                                                    \
     return encode_prefill_as<GG, CC>(g, layer, req, kv, tok_stride, kv_tokens, tok_begin, n_tok, \

@@ -241,7 +241,7 @@ __device__ inline void quad_min_mask(const uint32_t (&ra)[64], const uint32_t (&
 
 template <int G, int C>
 __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
-    const __grid_constant__ CUtensorMap tmap, Geo g, int layer, int req, int tok_begin, int n_tok,
+    const __grid_constant__ CUtensorMap tmap, Geo g, int layer0, int n_layers, int req, int tok_begin, int n_tok,
     int coded_offset, const __nv_bfloat16* __restrict__ cb, uint8_t* __restrict__ idx, int32_t* st) {
   using X = Enc<G, C>;
   constexpr int TC = X::TC, NGC = X::NGC, SBO = X::SBO;
@@ -303,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
   const int n_spans = g.d / kSpan;
   const int n_sets = 2 * g.nblk * g.H * n_spans;
   const int n_ranges = (n_tok + kItemTokens - 1) / kItemTokens;
-  const long n_items = (long)n_sets * n_ranges;
+  const long n_items = (long)n_sets * n_ranges * n_layers;    // layers outermost
 
   long T_glob = 0;          // raw tiles of the items before this one (this CTA)
   long J_glob = 0;          // group-tiles per team of the items before this one
@@ -312,7 +312,9 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
   long tiles_issued = 0;
 
   for (long item = blockIdx.x; item < n_items; item += gridDim.x) {
-    int cs = (int)(item / n_ranges);
+    const int lrel = (int)(item / ((long)n_sets * n_ranges));   // layer layer0 + lrel
+    const int layer = layer0 + lrel;
+    int cs = (int)(item % ((long)n_sets * n_ranges) / n_ranges);
     const int range = (int)(item % n_ranges);
     const int span = cs % n_spans; cs /= n_spans;
     const int h = cs % g.H; cs /= g.H;
@@ -380,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
           const uint32_t bar = smem_addr(&raw_full[stg]);
           mbar_expect_tx(bar, X::RAW);
           tma_load_3d(smem_addr(raw + stg * X::RAW), &tmap, h * g.d + span * kSpan, t_first + t * kTileTokens,
-                      kvi * g.T + blk * TC, bar);
+                      (lrel * 2 + kvi) * g.T + blk * TC, bar);
           tiles_issued = T + 1;
         }
       }
@@ -612,9 +614,11 @@ static cudaError_t encode_tc_as(const Geo& g, int layer, int req, const __nv_bfl
   using X = tc::Enc<G, C>;
   auto enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
+  // layer < 0: every layer in one launch; kv then holds the layers back to back
+  const int layer0 = layer < 0 ? 0 : layer, n_layers = layer < 0 ? g.L : 1;
   CUtensorMap map;
-  // dims: channels of a token row (H*d), tokens, (kv, step) planes
-  cuuint64_t dims[3] = {(cuuint64_t)g.H * g.d, (cuuint64_t)kv_tokens, (cuuint64_t)2 * g.T};
+  // dims: channels of a token row (H*d), tokens, (layer, kv, step) planes
+  cuuint64_t dims[3] = {(cuuint64_t)g.H * g.d, (cuuint64_t)kv_tokens, (cuuint64_t)n_layers * 2 * g.T};
   cuuint64_t strides[2] = {(cuuint64_t)tok_stride * 2, (cuuint64_t)tok_stride * kv_tokens * 2};
   cuuint32_t box[3] = {tc::kSpan, tc::kTileTokens, (cuuint32_t)X::TC};
   cuuint32_t estr[3] = {1, 1, 1};
@@ -637,9 +641,9 @@ static cudaError_t encode_tc_as(const Geo& g, int layer, int req, const __nv_bfl
     attr_set[dev] = true;
   }
   const long n_sets = 2L * g.nblk * g.H * (g.d / tc::kSpan);
-  const long items = n_sets * ((n_tok + tc::kItemTokens - 1) / tc::kItemTokens);
+  const long items = n_sets * ((n_tok + tc::kItemTokens - 1) / tc::kItemTokens) * n_layers;
   const int grid = (int)std::min<long>(items, n_sm[dev]);
-  tc::encode_tc_kernel<G, C><<<grid, tc::kThreads, X::SMEM, s>>>(map, g, layer, req, tok_begin, n_tok,
+  tc::encode_tc_kernel<G, C><<<grid, tc::kThreads, X::SMEM, s>>>(map, g, layer0, n_layers, req, tok_begin, n_tok,
                                                                   coded_offset, cb, idx, st);
   return cudaGetLastError();
 }

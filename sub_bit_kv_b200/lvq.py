@@ -143,11 +143,18 @@ def lvq_rope_table(cfg, lay, rope, stream=None):
 
 def lvq_encode_prefill(cfg, lay, layer, req, kv, tok_begin, n_tok, coded_offset, cb, idx, dev_status,
                        kv_tok_stride=None, stream=None):
-    """kv: bf16 [2][T][N][Hkv][d] of one layer and request (contiguous)."""
-    if kv.dim() != 5 or kv.shape[0] != 2 or kv.shape[1] != cfg.T:
+    """kv: bf16 [2][T][N][Hkv][d] of one layer and request (contiguous); with layer = -1
+    (every layer in one call) [n_layers][2][T][N][Hkv][d]."""
+    if layer == -1:
+        if kv.dim() != 6 or kv.shape[0] != cfg.n_layers:
+            raise ValueError("layer = -1 takes kv as [n_layers][2][T][N][Hkv][d]")
+        kv1 = kv[0]
+    else:
+        kv1 = kv
+    if kv1.dim() != 5 or kv1.shape[0] != 2 or kv1.shape[1] != cfg.T:
         raise ValueError("kv must be [2][T][N][Hkv][d]")
-    n_total = kv.shape[2]
-    stride = kv_tok_stride if kv_tok_stride is not None else kv.shape[3] * kv.shape[4]
+    n_total = kv1.shape[2]
+    stride = kv_tok_stride if kv_tok_stride is not None else kv1.shape[3] * kv1.shape[4]
     _check(lib().lvq_encode_prefill(
         ctypes.byref(cfg), ctypes.byref(lay), layer, req, _ptr(kv, "kv", torch.bfloat16), stride, n_total,
         tok_begin, n_tok, coded_offset, _ptr(cb, "cb", torch.bfloat16, lay.cb_bytes),

@@ -4,6 +4,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from oracle import lvq_oracle as O
 from sub_bit_kv_b200 import lvq, synth
@@ -137,3 +138,25 @@ def test_debug_fault_hook_host_side():
     assert e.value.status == lvq.LVQ_EINVAL
     lvq.lvq_debug_faults(1 << 10, 3)
     lvq.lvq_debug_faults(0, 0)
+
+
+def test_encode_prefill_layer_argument_on_the_host():
+    """layer = -1 (every layer in one call) passes the host checks -- on a machine without a
+    GPU it then stops at the device check -- while anything below -1 or past the last layer
+    is rejected first."""
+    import ctypes
+    w = synth.WORKLOADS["tiny"]
+    cfg = make_cfg(w)
+    lay = lvq.lvq_cache_layout(cfg)
+    L = lvq.lib()
+    fake = 1 << 20
+
+    def call(layer):
+        return L.lvq_encode_prefill(ctypes.byref(cfg), ctypes.byref(lay), layer, 0, fake,
+                                    w.n_kv_heads * w.head_dim, 64, 0, 64, 0, fake, fake, None, None)
+
+    assert call(-2) == lvq.LVQ_EINVAL
+    assert call(cfg.n_layers) == lvq.LVQ_EINVAL
+    if not torch.cuda.is_available():
+        assert call(-1) == lvq.LVQ_EDEVICE
+        assert call(0) == lvq.LVQ_EDEVICE

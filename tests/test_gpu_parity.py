@@ -75,6 +75,38 @@ def test_encode_prefill_matches_oracle(name, ntok, offset, extra):
 
 
 @pytest.mark.parametrize("name,extra", [
+    ("ouro14_g16_32k", {"n_kv_heads": 2, "n_q_heads": 2}),                 # tensor-core encoder, one launch
+    ("ouro14_tc2_64k", {"n_kv_heads": 2, "n_q_heads": 2}),                 # c = 8, two blocks per token
+    ("ouro14_g16_32k", {"Tc": 1, "n_kv_heads": 1, "n_q_heads": 1}),        # c = 16: direct form, per layer
+])
+def test_encode_prefill_all_layers_in_one_call(name, extra):
+    """layer = -1: the K/V of every layer back to back, encoded by one call; every layer's codes
+    equal the oracle's nearest entries (near-ties excepted), and none spill into another layer."""
+    w = _reduced(name, n_layers=3, **extra)
+    ntok, offset = 1500, 3
+    case = Hl.build_case(w, layers=3, ctx=[w.n_sink + ntok + offset + w.n_recent], coded=[ntok + offset],
+                         codes_from="none")
+    c = case.cache
+    kvs = [synth.loop_kv(w, layer, ntok, stream="enc-all") for layer in range(3)]   # [2][T][N][H][d] each
+    kv_all = torch.stack(kvs).cuda()                                                # [L][2][T][N][H][d]
+    c.idx.zero_()
+    lvq.lvq_encode_prefill(case.cfg, c.lay, -1, 0, kv_all, 0, ntok, offset, c.cb, c.idx, c.status)
+    torch.cuda.synchronize()
+    c.check_status()
+    for layer in range(3):
+        cb = Hl.f64(case.cb[layer])
+        x = Hl.f64(kvs[layer])
+        for kvi in range(2):
+            got = Hl.get_codes(c, layer, 0, kvi, offset, ntok).numpy()
+            assert not Hl.get_codes(c, layer, 0, kvi, 0, offset).numpy().any()   # slots before the offset
+            X = O.joint_vectors(x[kvi], w.Tc, w.G)
+            for blk in range(X.shape[0]):
+                for h in range(X.shape[2]):
+                    for g in range(X.shape[3]):
+                        check_codes(got[blk, :, h, g], X[blk, :, h, g], cb[kvi, blk, h, g])
+
+
+@pytest.mark.parametrize("name,extra", [
     ("ouro14_g16_32k", {"n_kv_heads": 2, "n_q_heads": 2}),     # G = 16, c = 4 (tensor-core encoder)
     ("ouro14_g32_b32", {"n_kv_heads": 2, "n_q_heads": 2}),     # G = 32, c = 8
 ])
