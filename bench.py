@@ -75,6 +75,8 @@ def parse(argv=None):
     ap.add_argument("--splits", type=int, default=0, help="split count (0: choose)")
     ap.add_argument("--workload", default=WORKLOAD, choices=list(DECODE_WORKLOADS) + [ENCODE_WORKLOAD])
     ap.add_argument("--no-encode", action="store_true", help="skip the one-layer prefill-encode measurement")
+    ap.add_argument("--pool", action="store_true",
+                    help="decode workloads: codes in a shared page pool behind an 8-token page table")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-sample", type=int, default=2,
                     help="units (head-attentions, or encode batches) per step of the reference (oracle) arm")
@@ -460,15 +462,32 @@ class Clocks:
                 "samples": len(rows)}
 
 
-def build_cache(w, lvq, synth, torch, extra_tokens: int, device, request_seed: int, max_splits: int = 128):
-    """Coded cache at the workload's per-request contexts, codes from the library's encoder."""
+POOL_BITE = 64      # pages a request takes from the pool at a time in pool mode (512 tokens)
+
+
+def build_cache(w, lvq, synth, torch, extra_tokens: int, device, request_seed: int, max_splits: int = 128,
+                pool: bool = False):
+    """Coded cache at the workload's per-request contexts, codes from the library's encoder.
+    pool: codes in a shared page pool; every request holds the pages of its context plus
+    extra_tokens, taken from the pool in round-robin bites of POOL_BITE pages (as requests that
+    grow side by side would take them), so its pages are runs of POOL_BITE consecutive ids."""
     ctx = synth.ctx_lengths(w)
     B = len(ctx)
+    coded = [c - w.n_sink - w.n_recent for c in ctx]
+    need = [(cd + extra_tokens + 7) // 8 for cd in coded]
     cfg = lvq.make_config(w.n_layers, w.n_kv_heads, w.n_q_heads, w.head_dim, w.T, w.Tc, w.G, w.n_sink,
-                          w.n_recent, B, max(ctx) + extra_tokens, max_splits=max_splits, rope_base=w.rope_base)
+                          w.n_recent, B, max(ctx) + extra_tokens, max_splits=max_splits, rope_base=w.rope_base,
+                          pool_pages=sum(need) if pool else 0)
     cache = lvq.CodedCache(cfg, device)
     lay = cache.lay
-    coded = [c - w.n_sink - w.n_recent for c in ctx]
+    if pool:
+        left = list(need)
+        while any(left):
+            for b in range(B):
+                k = min(POOL_BITE, left[b])
+                if k:
+                    cache.assign_pages(b, len(cache.pages[b]) + k)
+                    left[b] -= k
     cbv, sv, rv = cache.cb_view(), cache.sink_view(), cache.ring_view()
     for layer in range(w.n_layers):
         sc = synth.channel_scales(w, layer, device=device)
@@ -493,15 +512,23 @@ def build_cache(w, lvq, synth, torch, extra_tokens: int, device, request_seed: i
     return cfg, cache
 
 
+SPLIT_FIXED_TOKENS = 850    # a CTA's fixed cost (slices, prologue, merge) in coded tokens of work
+
+
 def choose_splits(w, n_sm: int) -> int:
-    """Splits per (request, head).  One CTA per SM: when the batch's heads fit in one wave,
-    as many splits as fill it; otherwise splits of about 6K coded tokens, which balance the
-    waves of a ragged batch against each CTA's fixed cost (measured on the 32-request
-    workload: 3-4 splits beat 1, 2 and 6)."""
+    """Splits per (request, head), one CTA per SM.  Requests of equal length: the count (up to
+    128) that minimises waves x (coded tokens per CTA + a CTA's fixed cost), the waves being
+    whole -- at the 32K workload 9 splits fill one wave (144 of 148 SMs; 10 would spill into a
+    second wave: 46 us against 27 us), at the 8-request 64K workload 8 splits give 7 nearly full
+    waves (327 us per launch, against 410 us for 1 split and 372 us for 7).  A ragged batch:
+    splits of about 6K coded tokens, which balance its waves against the fixed cost (measured on
+    the 32-request workload: 3 splits, 486 us, against 521 for 2 and 496 for 4)."""
     heads = w.batch * w.n_q_heads
-    if heads <= n_sm:
-        return max(1, min(128, n_sm // heads))
-    mean_ctx = w.ctx if w.ctx else (w.ctx_low + w.ctx_high) / 2
+    if w.ctx:
+        L = max(0, w.ctx - w.n_sink - w.n_recent)
+        cost = {ns: -(-heads * ns // n_sm) * (L / ns + SPLIT_FIXED_TOKENS) for ns in range(1, 129)}
+        return min(cost, key=lambda ns: (cost[ns], ns))
+    mean_ctx = (w.ctx_low + w.ctx_high) / 2
     return max(1, min(16, round(mean_ctx / 6144)))
 
 
@@ -665,7 +692,7 @@ def decode_arm(args, torch, dist, lvq, synth, world, rank, local, device):
     n_sm = torch.cuda.get_device_properties(device).multi_processor_count
     ns = args.splits or choose_splits(w, n_sm)
     cfg, cache = build_cache(w, lvq, synth, torch, TOKENS_PER_STEP * (replays + 4), device,
-                             replica_plan(rank, world, w.batch)["seed"], max_splits=max(128, ns))
+                             replica_plan(rank, world, w.batch)["seed"], max_splits=max(128, ns), pool=args.pool)
     lay = cache.lay
     B, Hq, d = w.batch, w.n_q_heads, w.head_dim
     if args.profile == "decode":
@@ -794,7 +821,8 @@ def decode_arm(args, torch, dist, lvq, synth, world, rank, local, device):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": decode_config(w, world, ns),
+        "config": dict(decode_config(w, world, ns), **({"codes": f"page pool, {POOL_BITE}-page bites"} if args.pool
+                                                         else {})),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak,
                      "traffic": decode_traffic() if args.workload == WORKLOAD else None,

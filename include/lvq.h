@@ -27,9 +27,10 @@
  *
  * Conventions for every entry point:
  *   - The caller owns every buffer (device memory unless stated).  The
- *     library allocates nothing and keeps no global state, apart from the
- *     fixed workspace of lvq_decode_attention_noalloc and the settings of the
- *     lvq_debug_faults test hook.
+ *     library allocates no device memory and keeps no global state, apart from
+ *     the fixed workspace of lvq_decode_attention_noalloc and the settings of
+ *     the lvq_debug_faults test hook; an lvq_pool is host bookkeeping the
+ *     caller creates and destroys.
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
  *     NULL is the legacy default stream).  Errors the host can see (bad
  *     config, null or misaligned pointer, out-of-range argument) return at
@@ -92,6 +93,18 @@ typedef struct {
   int32_t max_ctx;      /* longest context (tokens, including the query) */
   int32_t max_splits;   /* largest num_splits lvq_decode_attention accepts (<= 256) */
   float rope_base;      /* RoPE base (10000 for the Ouro-shaped workloads) */
+  /* Code storage.  pool_pages = 0: every (layer, block, request, head, K/V) has its own
+   * stream of max_pages pages.  pool_pages > 0: the requests share a pool of pool_pages
+   * 8-token pages per (layer, block, head, K/V), and page_table (device int32
+   * [max_batch][page_table_stride], see lvq_layout) maps request b's logical page i (its
+   * coded tokens 8i .. 8i+7) to a physical page, the same id in every (layer, block, head,
+   * K/V) pool; ids come from an lvq_pool.  A page table entry that a call needs but that is
+   * out of range (< 0 or >= pool_pages) sets LVQ_ECAPACITY in *dev_status; the decode then
+   * reads page 0 in its place (its output for that request is not meaningful) and the
+   * encoders skip the page. */
+  int32_t pool_pages;
+  int32_t reserved_;    /* must be 0 */
+  const int32_t* page_table;   /* device pointer; NULL when pool_pages = 0 */
 } lvq_config;
 
 /* Derived sizes and layouts.  All byte counts are totals for the whole
@@ -105,13 +118,17 @@ typedef struct {
   int32_t max_pages;    /* coded pages per (layer, block, request, head) */
   int32_t page_bytes;   /* bytes of one coded page of K or of V: n_g * 8 */
   int32_t rope_coarse;  /* rows of the coarse RoPE table (positions 8k) */
-  int32_t reserved;
+  int32_t page_table_stride;   /* int32 entries per request in the page table (pool mode) */
   /* uint8 codes, [layer][n_blk][B][Hkv][kv][page][n_g][8]: byte (g, j) of a
    * page holds group g's code of the page's token j (token n of the coded
    * region sits in page n/8 at j = n%8).  The K pages of a (layer, block,
-   * request, head) form one contiguous stream, followed by its V pages. */
+   * request, head) form one contiguous stream, followed by its V pages.
+   * Pool mode: [layer][n_blk][Hkv][kv][pool_pages][n_g][8], request b's logical page i
+   * at physical page page_table[b][i] (idx_strides: the 7 dimensions, then 0). */
   size_t idx_bytes;
   int64_t idx_strides[8];
+  /* device int32 [max_batch][page_table_stride]; 0 outside pool mode */
+  size_t page_table_bytes;
   /* bf16 logical codebooks, [layer][kv][n_blk][Hkv][n_g][256][G]; element
    * s*c + e of an entry is step s of the block, channel g*c + e. */
   size_t cb_bytes;
@@ -141,7 +158,9 @@ typedef struct {
 } lvq_layout;
 
 /* Sizes and strides for cfg.  Host arithmetic only: no CUDA call, usable
- * without a GPU.  Returns LVQ_EINVAL / LVQ_EUNSUPPORTED for a bad shape. */
+ * without a GPU.  Returns LVQ_EINVAL / LVQ_EUNSUPPORTED for a bad shape.  In
+ * pool mode cfg->page_table may still be NULL here (the layout gives the page
+ * table's size); every other call needs it. */
 LVQ_API lvq_status lvq_cache_layout(const lvq_config* cfg, lvq_layout* out);
 
 /* Message for a status code (static string, never NULL). */
@@ -212,7 +231,8 @@ LVQ_API lvq_status lvq_encode_prefill(const lvq_config* cfg, const lvq_layout* l
  * The packed codebooks and norms the decoder reads are not touched: call
  * lvq_pack_codebooks after the last iteration.  LVQ_EUNSUPPORTED where
  * (d/c) is not a multiple of 64/G or kv_tok_stride is not a multiple of 8
- * (the values are read by TMA); LVQ_EINVAL for out-of-range arguments, null
+ * (the values are read by TMA), and in pool mode (codebooks are built before
+ * serving, on per-request streams); LVQ_EINVAL for out-of-range arguments, null
  * or misaligned (16-byte) pointers.  Device-side: LVQ_ETIMEOUT in *dev_status
  * if a copy never lands (every wait is bounded). */
 LVQ_API lvq_status lvq_kmeans_update(const lvq_config* cfg, const lvq_layout* lay, int32_t layer,
@@ -274,6 +294,27 @@ LVQ_API lvq_status lvq_dequantize(const lvq_config* cfg, const lvq_layout* lay, 
                           int32_t step, int32_t req, int32_t kv, const uint8_t* idx,
                           const void* cbp, int32_t tok_begin, int32_t n_tok, void* out,
                           void* stream);
+
+/* Page pool bookkeeping (host memory only; device buffers stay the caller's).  "LoopVQ
+ * summary", "premises and limits": the cache is built from 8-token pages.  An lvq_pool hands
+ * out the physical page ids of a pool of n_pages pages (pool mode of lvq_config) to requests
+ * of any length and takes them back when a request ends; the caller writes the ids into the
+ * device page table.  Ids are handed out lowest first, so a request's pages tend to form
+ * runs of consecutive ids (the decode copies a run with one bulk copy).  Not thread-safe:
+ * one pool per host thread, or the caller's own lock. */
+typedef struct lvq_pool lvq_pool;
+/* n_pages >= 1; *out receives the pool (free it with lvq_pool_destroy).  LVQ_EINVAL for a
+ * bad argument. */
+LVQ_API lvq_status lvq_pool_create(int32_t n_pages, lvq_pool** out);
+LVQ_API void lvq_pool_destroy(lvq_pool* pool);
+/* n free page ids into ids[0..n), lowest first; LVQ_ECAPACITY (nothing taken) if fewer than
+ * n are free. */
+LVQ_API lvq_status lvq_pool_alloc(lvq_pool* pool, int32_t n, int32_t* ids);
+/* Returns n ids to the pool; LVQ_EINVAL (nothing returned) if an id is out of range, not
+ * currently handed out, or repeated. */
+LVQ_API lvq_status lvq_pool_free(lvq_pool* pool, const int32_t* ids, int32_t n);
+/* Free page ids (-1 for a null pool). */
+LVQ_API int32_t lvq_pool_available(const lvq_pool* pool);
 
 /* Decode attention without a caller-supplied workspace.  The pages have no
  * counterpart of this entry point: it exists for callers that cannot allocate

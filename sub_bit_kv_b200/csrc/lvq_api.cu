@@ -15,7 +15,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // LoopVQ shape rules ("LoopVQ summary", "how it differs": Tc divides T and G,
 // one code covers c = G/Tc channels of each step; "premises and limits": 8-bit
 // codes, K = 256, 8-token pages), then this build's kernel set.
-lvq_status check_cfg(const lvq_config* c) {
+lvq_status check_cfg(const lvq_config* c, bool need_table = true) {
   if (!c) return LVQ_EINVAL;
   if (c->n_layers < 1 || c->n_kv_heads < 1 || c->n_q_heads < 1 || c->head_dim < 2 || c->T < 1 ||
       c->Tc < 1 || c->G < 1 || c->n_sink < 0 || c->n_recent < 0 || c->max_batch < 1 ||
@@ -29,6 +29,11 @@ lvq_status check_cfg(const lvq_config* c) {
   if (!decode_supported(c->head_dim, cc) || !encode_supported(c->G, cc)) return LVQ_EUNSUPPORTED;
   if (c->max_splits > 256 || c->max_ctx > (1 << 28)) return LVQ_EUNSUPPORTED;
   if (c->n_sink + c->n_recent + kPage > decode_bf16_capacity(c->head_dim, cc)) return LVQ_EUNSUPPORTED;
+  // pool mode: a page table (16-byte aligned: the decode reads it in 16-byte pieces)
+  if (c->pool_pages < 0 || c->reserved_ != 0) return LVQ_EINVAL;
+  if (c->page_table && !aligned16(c->page_table)) return LVQ_EINVAL;
+  if (c->pool_pages == 0 && c->page_table) return LVQ_EINVAL;
+  if (need_table && c->pool_pages > 0 && !c->page_table) return LVQ_EINVAL;
   return LVQ_OK;
 }
 
@@ -48,6 +53,9 @@ Geo make_geo(const lvq_config* c) {
   g.page_bytes = g.ng * kPage;
   g.wait_iters = debug_wait_iters;
   g.fault = debug_fault;
+  g.pool = c->pool_pages;
+  g.pts = (g.P + 3) / 4 * 4;       // page-table row: whole 16-byte pieces
+  g.pt = c->page_table;
   return g;
 }
 
@@ -55,9 +63,16 @@ void fill_layout(const Geo& g, lvq_layout* o) {
   memset(o, 0, sizeof(*o));
   o->c = g.c; o->n_groups = g.ng; o->n_blocks = g.nblk; o->ring_tokens = g.R; o->max_pages = g.P;
   o->page_bytes = g.page_bytes; o->rope_coarse = g.RC;
-  const int64_t idims[8] = {g.L, g.nblk, g.B, g.H, 2, g.P, g.ng, kPage};
   int64_t st = 1;
-  for (int i = 7; i >= 0; --i) { o->idx_strides[i] = st; st *= idims[i]; }
+  if (g.pool == 0) {
+    const int64_t idims[8] = {g.L, g.nblk, g.B, g.H, 2, g.P, g.ng, kPage};
+    for (int i = 7; i >= 0; --i) { o->idx_strides[i] = st; st *= idims[i]; }
+  } else {
+    const int64_t idims[7] = {g.L, g.nblk, g.H, 2, g.pool, g.ng, kPage};
+    for (int i = 6; i >= 0; --i) { o->idx_strides[i] = st; st *= idims[i]; }
+    o->page_table_stride = g.pts;
+    o->page_table_bytes = (size_t)g.B * g.pts * 4;
+  }
   o->idx_bytes = (size_t)st;
   const int64_t cdims[7] = {g.L, 2, g.nblk, g.H, g.ng, kEntries, g.G};
   st = 1;
@@ -114,7 +129,7 @@ extern "C" {
 
 lvq_status lvq_cache_layout(const lvq_config* cfg, lvq_layout* out) {
   if (!out) return LVQ_EINVAL;
-  lvq_status s = check_cfg(cfg);
+  lvq_status s = check_cfg(cfg, false);   // the layout does not depend on the page table's address
   if (s != LVQ_OK) return s;
   fill_layout(make_geo(cfg), out);
   return LVQ_OK;
@@ -195,7 +210,7 @@ lvq_status lvq_kmeans_update(const lvq_config* cfg, const lvq_layout* lay, int32
   if (!kv || !cb || !idx || !aligned16(kv) || !aligned16(cb) || !aligned16(idx) ||
       (counts && !aligned16(counts)))
     return LVQ_EINVAL;
-  if (g.ng % (64 / g.G) != 0 || kv_tok_stride % 8 != 0) return LVQ_EUNSUPPORTED;
+  if (g.ng % (64 / g.G) != 0 || kv_tok_stride % 8 != 0 || g.pool) return LVQ_EUNSUPPORTED;
   if ((s = check_device()) != LVQ_OK) return s;
   return cuda_status(launch_kmeans_update(g, layer, req, static_cast<const __nv_bfloat16*>(kv), kv_tok_stride,
                                           kv_tokens, tok_begin, n_tok, coded_offset, idx,

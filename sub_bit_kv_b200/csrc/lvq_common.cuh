@@ -21,6 +21,9 @@ struct Geo {
   int page_bytes;
   long wait_iters;   // bound of every device-side wait (kWaitIters unless a test lowers it)
   int fault;         // test hook: kFault* bits, 0 in normal use
+  int pool;          // pool mode: physical pages per (layer, block, head, K/V); 0: per-request streams
+  int pts;           // page-table entries per request (pool mode)
+  const int32_t* pt; // device page table [B][pts] (pool mode)
 };
 // Test hook bits (lvq_debug_faults): a copy that is never issued, so that a bounded wait
 // runs out and the kernel reports LVQ_ETIMEOUT.
@@ -31,10 +34,26 @@ constexpr int kFaultKmeansDropTile = 2;    // k-means update: the first tile of 
 __host__ __device__ inline size_t idx_stream_off(const Geo& g, int layer, int blk, int b, int h, int kv) {
   return (((((size_t)layer * g.nblk + blk) * g.B + b) * g.H + h) * 2 + kv) * (size_t)g.P * g.page_bytes;
 }
-// byte offset of group grp's code of coded token n in that stream
-__host__ __device__ inline size_t idx_code_off(const Geo& g, int layer, int blk, int b, int h, int kv, int n,
-                                               int grp) {
-  return idx_stream_off(g, layer, blk, b, h, kv) + (size_t)(n >> 3) * g.page_bytes + grp * kPage + (n & 7);
+// Pool mode: byte offset of physical page 0 of the (layer, blk, h, kv) pool
+__host__ __device__ inline size_t idx_pool_off(const Geo& g, int layer, int blk, int h, int kv) {
+  return ((((size_t)layer * g.nblk + blk) * g.H + h) * 2 + kv) * (size_t)g.pool * g.page_bytes;
+}
+// Physical page of request b's logical page pg: itself outside pool mode, else the page
+// table's entry; -1 if the entry is out of range (the caller reports LVQ_ECAPACITY)
+__device__ inline int phys_page(const Geo& g, int b, int pg) {
+  if (g.pool == 0) return pg;
+  const int id = __ldg(g.pt + (size_t)b * g.pts + pg);
+  return id >= 0 && id < g.pool ? id : -1;
+}
+// byte offset of physical page `phys` of the code stream of (layer, blk, b, h, kv)
+__host__ __device__ inline size_t idx_page_off(const Geo& g, int layer, int blk, int b, int h, int kv, int phys) {
+  return g.pool ? idx_pool_off(g, layer, blk, h, kv) + (size_t)phys * g.page_bytes
+                : idx_stream_off(g, layer, blk, b, h, kv) + (size_t)phys * g.page_bytes;
+}
+// byte offset of group grp's code of coded token n (logical page n/8 is physical page phys)
+__host__ __device__ inline size_t idx_code_off(const Geo& g, int layer, int blk, int b, int h, int kv, int phys,
+                                               int n, int grp) {
+  return idx_page_off(g, layer, blk, b, h, kv, phys) + grp * kPage + (n & 7);
 }
 // element offset of the packed step slice [256][ng][c] of (layer, kv, blk, h, s)
 __host__ __device__ inline size_t cbp_slice_off(const Geo& g, int layer, int kv, int blk, int h, int s) {

@@ -539,8 +539,10 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
   const int n_stream = 2 * n_kchunks;            // per super-chunk: its K chunks, then its V chunks
   const int n_super = do_coded ? (n1 - n0 + X::NSC - 1) / X::NSC : 0;
   constexpr int CPS = X::NSC / kChunk;           // chunks per full super-chunk
-  const uint8_t* kstream = idx + idx_stream_off(g, layer, blk, b, h, 0);
-  const uint8_t* vstream = idx + idx_stream_off(g, layer, blk, b, h, 1);
+  // per-request streams: the K pages, then the V pages, of (layer, blk, b, h); pool mode: the pools
+  // of (layer, blk, h), the request's pages found through the page table
+  const uint8_t* kstream = idx + (g.pool ? idx_pool_off(g, layer, blk, h, 0) : idx_stream_off(g, layer, blk, b, h, 0));
+  const uint8_t* vstream = idx + (g.pool ? idx_pool_off(g, layer, blk, h, 1) : idx_stream_off(g, layer, blk, b, h, 1));
 
   // the V slice is needed only by the first contraction: the producer copies it once its bf16 share
   // (staged in the same area) is done
@@ -549,25 +551,79 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
     mbar_expect_tx(bv, X::KS);
     bulk_g2s(smem_addr(Vsm), cbp + cbp_slice_off(g, layer, 1, blk, h, s), X::KS, bv);
   };
-  // chunk `ci` of the stream: its first coded token and which half of the page stream it reads
-  auto issue_chunk = [&](int ci) {
-    if (DBG && (g.fault & kFaultDecodeDropChunk) && ci == 0) return;   // test hook: this copy never happens
+  // chunk `ci` of the stream: its first coded token and which half of the page stream it reads.
+  // Called by the whole producer warp.  Per-request streams: one bulk copy of the chunk's pages.
+  // Pool mode: lane l looks up the chunk's pages l and l + 32 in the page table, and every run of
+  // consecutive physical pages (within a half) is one bulk copy, issued by the lane at its start; an
+  // out-of-range entry is reported and page 0 copied in its place (so that the stage still fills).
+  // first coded token, pages and K/V side of chunk ci
+  auto chunk_geom = [&](int ci, int& c0, int& np, bool& is_v) {
     const int sc = ci / (2 * CPS), r = ci % (2 * CPS);
     const int nk = min(CPS, n_kchunks - sc * CPS);
-    const bool is_v = r >= nk;
-    const int c0 = n0 + (sc * CPS + (is_v ? r - nk : r)) * kChunk;
-    const int np = (min(n1, c0 + kChunk) - c0 + kPage - 1) / kPage;
+    is_v = r >= nk;
+    c0 = n0 + (sc * CPS + (is_v ? r - nk : r)) * kChunk;
+    np = (min(n1, c0 + kChunk) - c0 + kPage - 1) / kPage;
+  };
+  // pool mode: the page ids of the next chunk to issue are loaded one chunk ahead (lane l holds
+  // the chunk's pages l and l + 32) and range-checked only when they are used, so that the page
+  // table's latency overlaps the ring's wait instead of stalling the producer
+  int pf_ci = -1, pf_id[2] = {0, 0};
+  const int32_t* pt_row = g.pool ? g.pt + (size_t)b * g.pts : nullptr;
+  auto fetch_ids = [&](int ci) {
+    int c0, np;
+    bool v;
+    chunk_geom(ci, c0, np, v);
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int i = lane + 32 * hh;
+      pf_id[hh] = i < np ? __ldg(pt_row + c0 / kPage + i) : 0;
+    }
+    pf_ci = ci;
+  };
+  auto issue_chunk = [&](int ci) {
+    if (DBG && (g.fault & kFaultDecodeDropChunk) && ci == 0) return;   // test hook: this copy never happens
+    int c0, np;
+    bool is_v;
+    chunk_geom(ci, c0, np, is_v);
     const uint32_t bar = smem_addr(&bars[2 + ci % kStages]);
-    mbar_expect_tx(bar, np * X::PAGE);
-    bulk_g2s(smem_addr(ringb + (ci % kStages) * X::STAGE), (is_v ? vstream : kstream) + (size_t)(c0 / kPage) * X::PAGE,
-             np * X::PAGE, bar);
+    const uint32_t dst = smem_addr(ringb + (ci % kStages) * X::STAGE);
+    const uint8_t* src = is_v ? vstream : kstream;
+    if (lane == 0) mbar_expect_tx(bar, np * X::PAGE);
+    if (!g.pool) {
+      if (lane == 0) bulk_g2s(dst, src + (size_t)(c0 / kPage) * X::PAGE, np * X::PAGE, bar);
+      return;
+    }
+    if (pf_ci != ci) fetch_ids(ci);
+    const int ids[2] = {pf_id[0], pf_id[1]};
+    if (ci + 1 < n_stream) fetch_ids(ci + 1);      // in flight until the next chunk is issued
+    __syncwarp();                                   // the expected bytes are set before any copy lands
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int i = lane + 32 * hh;                 // page of the chunk
+      const int in_half = min(32, np - 32 * hh);    // pages of this half (may be <= 0)
+      int id = i < np ? ids[hh] : 0;
+      const bool bad = i < np && (id < 0 || id >= g.pool);
+      if (bad) {
+        set_status(st, LVQ_ECAPACITY);
+        id = 0;
+      }
+      const int prev = __shfl_up_sync(0xffffffffu, id, 1);
+      const bool prev_bad = __shfl_up_sync(0xffffffffu, bad, 1);
+      const bool start = i < np && (lane == 0 || bad || prev_bad || id != prev + 1);
+      const uint32_t starts = __ballot_sync(0xffffffffu, start);
+      if (start) {
+        const uint32_t later = lane < 31 ? starts >> (lane + 1) : 0u;
+        const int end = later ? lane + __ffs(later) : in_half;   // lane of the next run's start
+        bulk_g2s(dst + (uint32_t)i * X::PAGE, src + (size_t)id * X::PAGE, (uint32_t)(end - lane) * X::PAGE, bar);
+      }
+    }
   };
 
   // ---- prologue: the producer starts the first chunks; compute threads rotate the query (scaled so
   // that scores come out in log2 units) and clear the histogram
   const int nb = bad ? 0 : S_eff + recent;                 // bf16 tokens: [sink tokens, recent tokens]
   const int nbj = nb > j ? (nb - j + ns - 1) / ns : 0;    // this CTA's share: j, j + ns, ...
-  if (producer && lane == 0 && do_coded)
+  if (producer && do_coded)
     for (int ci = 0; ci < min(kStages, n_stream); ++ci) issue_chunk(ci);
   // a compute lane's RoPE factors at its first coded token, fetched now so that their latency
   // overlaps the prologue
@@ -599,15 +655,15 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
 
   if (do_coded) {
     if (producer) {
-      // ---- producer: the bf16 share, feeding the ring meanwhile (lane 0 issues every chunk whose
-      // stage its consumers have released); the V slice into the area the share used; then the
-      // rest of the chunks
+      // ---- producer: the bf16 share, feeding the ring meanwhile (every chunk whose stage its
+      // consumers have released, as lane 0 sees the stage); the V slice into the area the share
+      // used; then the rest of the chunks
       int ci_next = min(kStages, n_stream);
       auto service = [&]() {
-        if (lane == 0)
-          while (ci_next < n_stream &&
-                 mbar_test(smem_addr(&bars[2 + kStages + ci_next % kStages]), (ci_next / kStages - 1) & 1))
-            issue_chunk(ci_next++);
+        while (ci_next < n_stream &&
+               __shfl_sync(0xffffffffu, lane == 0 ? (int)mbar_test(smem_addr(&bars[2 + kStages + ci_next % kStages]),
+                                                                   (ci_next / kStages - 1) & 1) : 0, 0))
+          issue_chunk(ci_next++);
       };
       timed_out = bf16_share<D, C>(service, g, layer, step, b, h, j, ns, S_eff, Lc, nbj, sink, ring, rope, zq,
                                    smem + X::OFF_V, smem_addr(&bars[2 + 2 * kStages]), part_bf16, misc, wit);
@@ -615,16 +671,17 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
         issue_v_slice();
         misc[3] = 1;
       }
-      if (lane == 0) {
+      {
         int ci = ci_next;
         for (; ci < n_stream; ++ci) {
-          if (!mbar_wait(smem_addr(&bars[2 + kStages + ci % kStages]), (ci / kStages - 1) & 1, wit)) {
+          if (__any_sync(0xffffffffu,
+                         !mbar_wait(smem_addr(&bars[2 + kStages + ci % kStages]), (ci / kStages - 1) & 1, wit))) {
             timed_out = true;
             break;
           }
           issue_chunk(ci);
         }
-        misc[2] = ci;
+        if (lane == 0) misc[2] = ci;
       }
     } else {
       // ---- compute warps

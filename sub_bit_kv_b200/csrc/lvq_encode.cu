@@ -19,7 +19,7 @@ template <int G, int C>
 __global__ void __launch_bounds__(kEncThreads) encode_prefill_kernel(
     Geo g, int layer, int req, const __nv_bfloat16* __restrict__ kv, int64_t tok_stride, int kv_tokens,
     int tok_begin, int n_tok, int coded_offset, const __nv_bfloat16* __restrict__ cb,
-    uint8_t* __restrict__ idx) {
+    uint8_t* __restrict__ idx, int32_t* st) {
   constexpr int TC = G / C;
   __shared__ float cbs[kEntries * G];   // fp32 copies of the bf16 entries (exact)
   int cid = blockIdx.y;
@@ -60,17 +60,22 @@ __global__ void __launch_bounds__(kEncThreads) encode_prefill_kernel(
     if (acc < best) { best = acc; bk = k; }
   }
   const int cn = coded_offset + local;
-  idx[idx_code_off(g, layer, blk, req, h, kvi, cn, grp)] = (uint8_t)bk;
+  const int phys = phys_page(g, req, cn >> 3);
+  if (phys < 0) {
+    set_status(st, LVQ_ECAPACITY);
+    return;
+  }
+  idx[idx_code_off(g, layer, blk, req, h, kvi, phys, cn, grp)] = (uint8_t)bk;
 }
 
 template <int G, int C>
 static cudaError_t encode_prefill_as(const Geo& g, int layer, int req, const __nv_bfloat16* kv,
                                      int64_t tok_stride, int kv_tokens, int tok_begin, int n_tok,
                                      int coded_offset, const __nv_bfloat16* cb, uint8_t* idx,
-                                     cudaStream_t s) {
+                                     int32_t* st, cudaStream_t s) {
   dim3 grid((n_tok + kEncThreads - 1) / kEncThreads, 2 * g.nblk * g.H * g.ng);
   encode_prefill_kernel<G, C><<<grid, kEncThreads, 0, s>>>(g, layer, req, kv, tok_stride, kv_tokens,
-                                                            tok_begin, n_tok, coded_offset, cb, idx);
+                                                            tok_begin, n_tok, coded_offset, cb, idx, st);
   return cudaGetLastError();
 }
 
@@ -82,7 +87,6 @@ cudaError_t launch_encode_prefill(const Geo& g, int layer, int req, const __nv_b
                                   int64_t tok_stride, int kv_tokens, int tok_begin, int n_tok,
                                   int coded_offset, const __nv_bfloat16* cb, uint8_t* idx,
                                   int32_t* st, cudaStream_t s) {
-  (void)st;
   if (n_tok == 0) return cudaSuccess;
   if (layer < 0) {   // every layer: kv holds the layers back to back, one launch each
     const int64_t layer_stride = (int64_t)2 * g.T * kv_tokens * tok_stride;
@@ -96,7 +100,7 @@ cudaError_t launch_encode_prefill(const Geo& g, int layer, int req, const __nv_b
 #define LVQ_ENC(GG, CC)                                                                          \
   if (g.G == GG && g.c == CC)                                                                    \
     return encode_prefill_as<GG, CC>(g, layer, req, kv, tok_stride, kv_tokens, tok_begin, n_tok, \
-                                     coded_offset, cb, idx, s);
+                                     coded_offset, cb, idx, st, s);
   LVQ_ENC(16, 4) LVQ_ENC(16, 8) LVQ_ENC(16, 16) LVQ_ENC(32, 4) LVQ_ENC(32, 8) LVQ_ENC(32, 16)
 #undef LVQ_ENC
   return cudaErrorInvalidValue;
@@ -360,8 +364,11 @@ __global__ void __launch_bounds__(PageEnc<G, C>::NW * 32, 1) encode_page_kernel(
       }
       if (r8 == 0) {                            // this lane's two tokens (coded_len need not be a multiple of 8)
         const int n = coded + 2 * q;
-        idx[idx_code_off(g, layer, blk, b, h, kvi, n, grp)] = (uint8_t)k0;
-        idx[idx_code_off(g, layer, blk, b, h, kvi, n + 1, grp)] = (uint8_t)k1;
+        // the 8 tokens may straddle two logical pages (coded_len need not be a multiple of 8)
+        const int p0 = phys_page(g, b, n >> 3), p1 = phys_page(g, b, (n + 1) >> 3);
+        if (p0 < 0 || p1 < 0) set_status(st, LVQ_ECAPACITY);
+        if (p0 >= 0) idx[idx_code_off(g, layer, blk, b, h, kvi, p0, n, grp)] = (uint8_t)k0;
+        if (p1 >= 0) idx[idx_code_off(g, layer, blk, b, h, kvi, p1, n + 1, grp)] = (uint8_t)k1;
       }
     }
     fence_proxy_async_shared();                 // this warp's reads of the slot precede its refill

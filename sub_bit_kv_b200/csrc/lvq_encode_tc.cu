@@ -324,7 +324,6 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
     const int t_last = min(tok_begin + n_tok, t_first + kItemTokens);
     const int n_tiles = (t_last - t_first + kTileTokens - 1) / kTileTokens;
     const int n_j = n_tiles * NGC / 2;              // group-tiles per team
-    uint8_t* const idx_item = idx + idx_stream_off(g, layer, blk, req, h, kvi);
 
     // every role has finished the previous item: its MMAs completed (the teams waited for
     // each), its raw tiles landed (the teams waited for each)
@@ -555,7 +554,11 @@ __global__ void __launch_bounds__(kThreads, 1) encode_tc_kernel(
             code = bk;
           }
           const int cn = coded_offset + (t0 + row - tok_begin);
-          idx_item[(size_t)(cn >> 3) * g.page_bytes + (span * NGC + gi) * kPage + (cn & 7)] = (uint8_t)code;
+          const int phys = phys_page(g, req, cn >> 3);
+          if (phys >= 0)
+            idx[idx_code_off(g, layer, blk, req, h, kvi, phys, cn, span * NGC + gi)] = (uint8_t)code;
+          else
+            set_status(st, LVQ_ECAPACITY);
         }
         // the last group-tile of raw tile t for this team: the stage may be refilled
         if (gi + 2 >= NGC) {

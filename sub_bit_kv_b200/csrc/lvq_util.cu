@@ -71,7 +71,8 @@ __global__ void dequant_kernel(Geo g, int layer, int step, int req, int kv, cons
     int h = (int)((i / g.d) % g.H);
     int n = tok_begin + (int)(i / ((size_t)g.d * g.H));
     int grp = ch / g.c, e = ch % g.c;
-    const int code = idx[idx_code_off(g, layer, blk, req, h, kv, n, grp)];
+    const int phys = phys_page(g, req, n >> 3);
+    const int code = phys < 0 ? 0 : idx[idx_code_off(g, layer, blk, req, h, kv, phys, n, grp)];
     const __nv_bfloat16* slice = cbp + cbp_slice_off(g, layer, kv, blk, h, s);
     out[i] = slice[((size_t)code * g.ng + grp) * g.c + e];
   }

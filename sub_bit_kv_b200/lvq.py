@@ -28,13 +28,15 @@ class LvqError(RuntimeError):
 class lvq_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "n_layers", "n_kv_heads", "n_q_heads", "head_dim", "T", "Tc", "G", "K", "n_sink", "n_recent",
-        "page_tokens", "max_batch", "max_ctx", "max_splits")] + [("rope_base", ctypes.c_float)]
+        "page_tokens", "max_batch", "max_ctx", "max_splits")] + [("rope_base", ctypes.c_float)] + [
+        ("pool_pages", ctypes.c_int32), ("reserved_", ctypes.c_int32), ("page_table", ctypes.c_void_p)]
 
 
 class lvq_layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
-        "c", "n_groups", "n_blocks", "ring_tokens", "max_pages", "page_bytes", "rope_coarse", "reserved")] + [
-        ("idx_bytes", ctypes.c_size_t), ("idx_strides", ctypes.c_int64 * 8),
+        "c", "n_groups", "n_blocks", "ring_tokens", "max_pages", "page_bytes", "rope_coarse",
+        "page_table_stride")] + [
+        ("idx_bytes", ctypes.c_size_t), ("idx_strides", ctypes.c_int64 * 8), ("page_table_bytes", ctypes.c_size_t),
         ("cb_bytes", ctypes.c_size_t), ("cb_strides", ctypes.c_int64 * 7),
         ("cbp_bytes", ctypes.c_size_t), ("cbp_strides", ctypes.c_int64 * 8),
         ("cb_norm_bytes", ctypes.c_size_t),
@@ -63,6 +65,11 @@ _SIGS = {
     "lvq_debug_faults": [ctypes.c_int64, _I32],
     "lvq_decode_attention_noalloc": [ctypes.POINTER(lvq_config), ctypes.POINTER(lvq_layout), _I32, _I32, _I32,
                                      _P, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P, _P],
+    "lvq_pool_create": [_I32, ctypes.POINTER(_P)],
+    "lvq_pool_destroy": [_P],
+    "lvq_pool_alloc": [_P, _I32, ctypes.POINTER(_I32)],
+    "lvq_pool_free": [_P, ctypes.POINTER(_I32), _I32],
+    "lvq_pool_available": [_P],
 }
 EXPORTED = tuple(_SIGS)
 
@@ -79,7 +86,7 @@ def lib():
         for name, args in _SIGS.items():
             fn = getattr(h, name)
             fn.argtypes = args
-            fn.restype = ctypes.c_char_p if name == "lvq_status_string" else ctypes.c_int
+            fn.restype = {"lvq_status_string": ctypes.c_char_p, "lvq_pool_destroy": None}.get(name, ctypes.c_int)
         _lib = h
     return _lib
 
@@ -94,9 +101,38 @@ def _check(s: int, where: str):
 
 
 def make_config(n_layers, n_kv_heads, n_q_heads, head_dim, T, Tc, G, n_sink, n_recent, max_batch, max_ctx,
-                max_splits=64, rope_base=10000.0, K=256, page_tokens=8) -> lvq_config:
+                max_splits=64, rope_base=10000.0, K=256, page_tokens=8, pool_pages=0) -> lvq_config:
+    """pool_pages > 0: pool mode (CodedCache allocates the page table and sets page_table)."""
     return lvq_config(n_layers, n_kv_heads, n_q_heads, head_dim, T, Tc, G, K, n_sink, n_recent, page_tokens,
-                      max_batch, max_ctx, max_splits, rope_base)
+                      max_batch, max_ctx, max_splits, rope_base, pool_pages, 0, None)
+
+
+class PagePool:
+    """The library's host-side page allocator (lvq_pool): physical page ids of a pool, handed
+    out lowest first and taken back when a request ends."""
+
+    def __init__(self, n_pages: int):
+        h = _P()
+        _check(lib().lvq_pool_create(int(n_pages), ctypes.byref(h)), "lvq_pool_create")
+        self._h = h
+
+    def alloc(self, n: int) -> list:
+        ids = (_I32 * max(1, n))()
+        _check(lib().lvq_pool_alloc(self._h, int(n), ids), "lvq_pool_alloc")
+        return list(ids[:n])
+
+    def free(self, ids) -> None:
+        arr = (_I32 * max(1, len(ids)))(*ids)
+        _check(lib().lvq_pool_free(self._h, arr, len(ids)), "lvq_pool_free")
+
+    def available(self) -> int:
+        return int(lib().lvq_pool_available(self._h))
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and _lib is not None:
+            _lib.lvq_pool_destroy(h)
+            self._h = None
 
 
 def lvq_cache_layout(cfg: lvq_config) -> lvq_layout:
@@ -256,6 +292,32 @@ class CodedCache:
         self.ctx_len = torch.zeros(cfg.max_batch, dtype=torch.int32, device=dev)
         self.coded_len = torch.zeros(cfg.max_batch, dtype=torch.int32, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.pool = None
+        if cfg.pool_pages > 0:
+            # pool mode: the page table (every entry unassigned) and the host allocator; the
+            # config carries the table's device address from here on
+            self.page_table = torch.full((lay.page_table_bytes // 4,), -1, dtype=torch.int32, device=dev)
+            cfg.page_table = self.page_table.data_ptr()
+            self.pool = PagePool(cfg.pool_pages)
+            self.pages = [[] for _ in range(cfg.max_batch)]       # host copy: physical page of logical page i
+
+    # pool mode: pages of a request
+    def assign_pages(self, b: int, n_pages: int) -> list:
+        """Makes request b hold at least n_pages logical pages (new ones from the pool) and writes
+        its page-table row.  Returns the request's physical pages."""
+        have = self.pages[b]
+        if n_pages > len(have):
+            have += self.pool.alloc(n_pages - len(have))
+            row = torch.tensor(have, dtype=torch.int32)
+            self.page_table[b * self.lay.page_table_stride: b * self.lay.page_table_stride + len(have)].copy_(row)
+        return list(have)
+
+    def release(self, b: int) -> None:
+        """Request b ends: its pages go back to the pool and its page-table row is cleared."""
+        if self.pages[b]:
+            self.pool.free(self.pages[b])
+            self.pages[b] = []
+            self.page_table[b * self.lay.page_table_stride:(b + 1) * self.lay.page_table_stride].fill_(-1)
 
     # shaped views of the caller-owned buffers (layouts from lvq_cache_layout)
     def cb_view(self):
@@ -272,6 +334,8 @@ class CodedCache:
 
     def idx_view(self):
         c, l = self.cfg, self.lay
+        if c.pool_pages > 0:       # [layer][n_blk][Hkv][kv][pool page][n_g][8]
+            return self.idx.view(c.n_layers, l.n_blocks, c.n_kv_heads, 2, c.pool_pages, l.n_groups, 8)
         return self.idx.view(c.n_layers, l.n_blocks, c.max_batch, c.n_kv_heads, 2, l.max_pages, l.n_groups, 8)
 
     def check_status(self, where="device"):

@@ -21,7 +21,8 @@ def built():
 
 def declared_functions():
     text = open(HEADER).read()
-    return sorted(set(re.findall(r"^\s*(?:LVQ_API\s+)?(?:lvq_status|const char\*)\s+(lvq_\w+)\s*\(", text, re.M)))
+    return sorted(set(re.findall(r"^\s*(?:LVQ_API\s+)?(?:lvq_status|const char\*|void|int32_t)\s+(lvq_\w+)\s*\(",
+                                 text, re.M)))
 
 
 def test_exports_every_declared_symbol():
@@ -160,3 +161,52 @@ def test_encode_prefill_layer_argument_on_the_host():
     if not torch.cuda.is_available():
         assert call(-1) == lvq.LVQ_EDEVICE
         assert call(0) == lvq.LVQ_EDEVICE
+
+
+def test_pool_allocator_hands_out_lowest_ids_and_takes_them_back():
+    pool = lvq.PagePool(10)
+    assert pool.available() == 10
+    assert pool.alloc(4) == [0, 1, 2, 3]
+    assert pool.alloc(3) == [4, 5, 6]
+    pool.free([1, 2])
+    assert pool.available() == 5
+    assert pool.alloc(2) == [1, 2]                  # lowest first: runs of consecutive ids
+    with pytest.raises(lvq.LvqError) as e:
+        pool.alloc(4)                               # only 3 left: nothing taken
+    assert e.value.status == lvq.LVQ_ECAPACITY and pool.available() == 3
+    for bad in ([10], [-1], [7], [0, 0]):           # out of range, out of range, free, repeated
+        with pytest.raises(lvq.LvqError) as e:
+            pool.free(bad)
+        assert e.value.status == lvq.LVQ_EINVAL
+    assert pool.available() == 3                    # all or nothing
+    pool.free([0, 3, 4])
+    assert pool.available() == 6
+
+
+def test_pool_layout_closed_forms_and_table_checks():
+    """Pool mode: codes live in pool_pages pages per (layer, block, head, K/V); the page table is
+    [max_batch][stride] with the stride the request's page capacity rounded up to 4."""
+    import ctypes
+    w = synth.WORKLOADS["ouro14_tc2_64k"]
+    cfg = make_cfg(w, n_layers=2, max_batch=3, max_ctx=1000)
+    plain = lvq.lvq_cache_layout(cfg)
+    cfg.pool_pages = 77
+    lay = lvq.lvq_cache_layout(cfg)                 # the table's address is not needed for the layout
+    c, ng, nblk = O.geometry(w.head_dim, w.T, w.Tc, w.G)
+    assert lay.idx_bytes == 2 * nblk * w.n_kv_heads * 2 * 77 * ng * 8
+    assert lay.page_table_stride == (plain.max_pages + 3) // 4 * 4
+    assert lay.page_table_bytes == 3 * lay.page_table_stride * 4
+    assert list(lay.idx_strides)[4:] == [ng * 8, 8, 1, 0]
+    assert plain.page_table_bytes == 0 and plain.page_table_stride == 0
+    L = lvq.lib()
+    # any call that reads or writes codes needs the table (host check, before any device work)
+    st = L.lvq_decode_attention(ctypes.byref(cfg), ctypes.byref(lay), 0, 0, 1, *([None] * 8), 1,
+                                None, None, None, None, None, None)
+    assert st == lvq.LVQ_EINVAL
+    cfg.page_table = 1 << 20
+    fake = 1 << 20
+    st = L.lvq_kmeans_update(ctypes.byref(cfg), ctypes.byref(lay), 0, 0, fake, w.n_kv_heads * w.head_dim, 64, 0,
+                             64, 0, fake, fake, None, None, None)
+    assert st == lvq.LVQ_EUNSUPPORTED                # codebooks are built on per-request streams
+    cfg.page_table = (1 << 20) + 4                   # misaligned table
+    assert lvq.lib().lvq_cache_layout(ctypes.byref(cfg), ctypes.byref(lvq.lvq_layout())) == lvq.LVQ_EINVAL

@@ -56,7 +56,7 @@ def test_decode_bytes_batch_counts_slices_once():
 def test_choose_splits():
     ws = synth.WORKLOADS
     assert bench.choose_splits(ws["ouro14_g16_32k"], 148) == 9         # 16 heads fill one wave
-    assert bench.choose_splits(ws["ouro14_tc2_64k"], 148) == 1         # 128 heads already fill it
+    assert bench.choose_splits(ws["ouro14_tc2_64k"], 148) == 8         # 1024 CTAs: 7 nearly full waves
     assert bench.choose_splits(ws["ouro14_g32_b32"], 148) == 3         # 512 heads: ~6K-token splits
     tiny = dataclasses.replace(ws["tiny"], batch=1)
     assert bench.choose_splits(tiny, 148) == 128                        # capped
