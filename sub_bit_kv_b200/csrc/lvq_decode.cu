@@ -464,8 +464,9 @@ __device__ bool bf16_share(Service& service, const Geo& g, int layer, int step, 
 }
 
 // DBG: the instantiation used while the test hook is active (its wait bound and fault bits
-// come from the geometry); the normal one keeps the constant bound.
-template <int D, int C, bool DBG>
+// come from the geometry); the normal ones keep the constant bound.  PM: 0 per-request code
+// streams, 1 pool mode, -1 either (read from the geometry; the test-hook instantiation).
+template <int D, int C, bool DBG, int PM>
 __global__ void __launch_bounds__(kThr, 1) decode_kernel(
     Geo g, int layer, int step, const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ ctx_len,
     const int32_t* __restrict__ coded_len, const __nv_bfloat16* __restrict__ sink,
@@ -475,6 +476,7 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
     int32_t* st) {
   using X = Dec<D, C>;
   const long wit = DBG ? g.wait_iters : kWaitIters;   // bound of every wait
+  const bool pool = PM < 0 ? g.pool != 0 : PM != 0;
   constexpr int F = X::F, NG = X::NG, TQ = X::TQ, NPAIR = X::NPAIR, NREP = X::NREP;
   extern __shared__ __align__(1024) unsigned char smem[];
   unsigned char* Ks = smem;
@@ -541,8 +543,8 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
   constexpr int CPS = X::NSC / kChunk;           // chunks per full super-chunk
   // per-request streams: the K pages, then the V pages, of (layer, blk, b, h); pool mode: the pools
   // of (layer, blk, h), the request's pages found through the page table
-  const uint8_t* kstream = idx + (g.pool ? idx_pool_off(g, layer, blk, h, 0) : idx_stream_off(g, layer, blk, b, h, 0));
-  const uint8_t* vstream = idx + (g.pool ? idx_pool_off(g, layer, blk, h, 1) : idx_stream_off(g, layer, blk, b, h, 1));
+  const uint8_t* kstream = idx + (pool ? idx_pool_off(g, layer, blk, h, 0) : idx_stream_off(g, layer, blk, b, h, 0));
+  const uint8_t* vstream = idx + (pool ? idx_pool_off(g, layer, blk, h, 1) : idx_stream_off(g, layer, blk, b, h, 1));
 
   // the V slice is needed only by the first contraction: the producer copies it once its bf16 share
   // (staged in the same area) is done
@@ -551,11 +553,6 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
     mbar_expect_tx(bv, X::KS);
     bulk_g2s(smem_addr(Vsm), cbp + cbp_slice_off(g, layer, 1, blk, h, s), X::KS, bv);
   };
-  // chunk `ci` of the stream: its first coded token and which half of the page stream it reads.
-  // Called by the whole producer warp.  Per-request streams: one bulk copy of the chunk's pages.
-  // Pool mode: lane l looks up the chunk's pages l and l + 32 in the page table, and every run of
-  // consecutive physical pages (within a half) is one bulk copy, issued by the lane at its start; an
-  // out-of-range entry is reported and page 0 copied in its place (so that the stage still fills).
   // first coded token, pages and K/V side of chunk ci
   auto chunk_geom = [&](int ci, int& c0, int& np, bool& is_v) {
     const int sc = ci / (2 * CPS), r = ci % (2 * CPS);
@@ -568,7 +565,7 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
   // the chunk's pages l and l + 32) and range-checked only when they are used, so that the page
   // table's latency overlaps the ring's wait instead of stalling the producer
   int pf_ci = -1, pf_id[2] = {0, 0};
-  const int32_t* pt_row = g.pool ? g.pt + (size_t)b * g.pts : nullptr;
+  const int32_t* pt_row = pool ? g.pt + (size_t)b * g.pts : nullptr;
   auto fetch_ids = [&](int ci) {
     int c0, np;
     bool v;
@@ -580,6 +577,11 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
     }
     pf_ci = ci;
   };
+  // issue chunk ci.  Per-request streams: lane 0 alone, one bulk copy of the chunk's pages.  Pool
+  // mode: the whole producer warp; lane l looks up the chunk's pages l and l + 32 in the page
+  // table, and every run of consecutive physical pages (within a half) is one bulk copy, issued by
+  // the lane at its start; an out-of-range entry is reported and page 0 copied in its place (so
+  // that the stage still fills).
   auto issue_chunk = [&](int ci) {
     if (DBG && (g.fault & kFaultDecodeDropChunk) && ci == 0) return;   // test hook: this copy never happens
     int c0, np;
@@ -589,8 +591,8 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
     const uint32_t dst = smem_addr(ringb + (ci % kStages) * X::STAGE);
     const uint8_t* src = is_v ? vstream : kstream;
     if (lane == 0) mbar_expect_tx(bar, np * X::PAGE);
-    if (!g.pool) {
-      if (lane == 0) bulk_g2s(dst, src + (size_t)(c0 / kPage) * X::PAGE, np * X::PAGE, bar);
+    if (!pool) {
+      bulk_g2s(dst, src + (size_t)(c0 / kPage) * X::PAGE, np * X::PAGE, bar);
       return;
     }
     if (pf_ci != ci) fetch_ids(ci);
@@ -623,7 +625,7 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
   // that scores come out in log2 units) and clear the histogram
   const int nb = bad ? 0 : S_eff + recent;                 // bf16 tokens: [sink tokens, recent tokens]
   const int nbj = nb > j ? (nb - j + ns - 1) / ns : 0;    // this CTA's share: j, j + ns, ...
-  if (producer && do_coded)
+  if (producer && do_coded && (pool || lane == 0))
     for (int ci = 0; ci < min(kStages, n_stream); ++ci) issue_chunk(ci);
   // a compute lane's RoPE factors at its first coded token, fetched now so that their latency
   // overlaps the prologue
@@ -657,13 +659,19 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
     if (producer) {
       // ---- producer: the bf16 share, feeding the ring meanwhile (every chunk whose stage its
       // consumers have released, as lane 0 sees the stage); the V slice into the area the share
-      // used; then the rest of the chunks
+      // used; then the rest of the chunks.  The ring is fed by lane 0 (per-request streams) or by
+      // the whole warp (pool mode).
       int ci_next = min(kStages, n_stream);
+      auto stage_free = [&](int ci) {
+        return mbar_test(smem_addr(&bars[2 + kStages + ci % kStages]), (ci / kStages - 1) & 1);
+      };
       auto service = [&]() {
-        while (ci_next < n_stream &&
-               __shfl_sync(0xffffffffu, lane == 0 ? (int)mbar_test(smem_addr(&bars[2 + kStages + ci_next % kStages]),
-                                                                   (ci_next / kStages - 1) & 1) : 0, 0))
-          issue_chunk(ci_next++);
+        if (pool) {
+          while (ci_next < n_stream && __shfl_sync(0xffffffffu, lane == 0 ? (int)stage_free(ci_next) : 0, 0))
+            issue_chunk(ci_next++);
+        } else if (lane == 0) {
+          while (ci_next < n_stream && stage_free(ci_next)) issue_chunk(ci_next++);
+        }
       };
       timed_out = bf16_share<D, C>(service, g, layer, step, b, h, j, ns, S_eff, Lc, nbj, sink, ring, rope, zq,
                                    smem + X::OFF_V, smem_addr(&bars[2 + 2 * kStages]), part_bf16, misc, wit);
@@ -671,11 +679,12 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
         issue_v_slice();
         misc[3] = 1;
       }
-      {
+      if (pool || lane == 0) {
         int ci = ci_next;
         for (; ci < n_stream; ++ci) {
-          if (__any_sync(0xffffffffu,
-                         !mbar_wait(smem_addr(&bars[2 + kStages + ci % kStages]), (ci / kStages - 1) & 1, wit))) {
+          bool ok = mbar_wait(smem_addr(&bars[2 + kStages + ci % kStages]), (ci / kStages - 1) & 1, wit);
+          if (pool) ok = __all_sync(0xffffffffu, ok);
+          if (!ok) {
             timed_out = true;
             break;
           }
@@ -955,12 +964,11 @@ static cudaError_t decode_as(const Geo& g, int layer, int step, int batch, const
   cudaError_t ge = cudaGetDevice(&dev);
   if (ge != cudaSuccess) return ge;
   if (dev < 0 || dev >= kMaxDevices || !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, C, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Dec<D, C>::SMEM);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(decode_kernel<D, C, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Dec<D, C>::SMEM);
-    if (e != cudaSuccess) return e;
+    for (const void* fn : {(const void*)decode_kernel<D, C, false, 0>, (const void*)decode_kernel<D, C, false, 1>,
+                           (const void*)decode_kernel<D, C, true, -1>}) {
+      const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, Dec<D, C>::SMEM);
+      if (e != cudaSuccess) return e;
+    }
     if (dev >= 0 && dev < kMaxDevices) attr_set[dev] = true;
   }
   const bool dbg = g.fault != 0 || g.wait_iters != kWaitIters;   // the test hook is active
@@ -975,10 +983,13 @@ static cudaError_t decode_as(const Geo& g, int layer, int step, int batch, const
   lc.attrs = attr;
   lc.numAttrs = 1;
   if (dbg)
-    return cudaLaunchKernelEx(&lc, decode_kernel<D, C, true>, g, layer, step, q, ctx_len, coded_len, sink, ring,
+    return cudaLaunchKernelEx(&lc, decode_kernel<D, C, true, -1>, g, layer, step, q, ctx_len, coded_len, sink, ring,
                               idx, cbp, rope, ns, ws, out, lse, split_lse, st);
-  return cudaLaunchKernelEx(&lc, decode_kernel<D, C, false>, g, layer, step, q, ctx_len, coded_len, sink, ring, idx,
-                            cbp, rope, ns, ws, out, lse, split_lse, st);
+  if (g.pool)
+    return cudaLaunchKernelEx(&lc, decode_kernel<D, C, false, 1>, g, layer, step, q, ctx_len, coded_len, sink, ring,
+                              idx, cbp, rope, ns, ws, out, lse, split_lse, st);
+  return cudaLaunchKernelEx(&lc, decode_kernel<D, C, false, 0>, g, layer, step, q, ctx_len, coded_len, sink, ring,
+                            idx, cbp, rope, ns, ws, out, lse, split_lse, st);
 }
 
 // Sink + recent-window tokens one call can take: a CTA keeps the scores of its
