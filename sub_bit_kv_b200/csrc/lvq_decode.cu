@@ -276,6 +276,29 @@ __device__ inline float run_scores(const Lane<D, C>& L, const unsigned char* Ks,
   return acc[0];
 }
 
+// A request's counters and the coded token range [n0, n1) of split j of ns (one split per
+// ceil(Lc / ns) tokens, rounded up to 32).  `bad`: counters outside the cache's capacity.
+struct SplitRange {
+  bool bad;
+  int S_eff, recent, n0, n1;
+};
+__device__ inline SplitRange split_range(const Geo& g, int ctx, int Lc, int j, int ns) {
+  SplitRange r;
+  r.S_eff = min(g.S, max(ctx, 0));
+  r.recent = ctx - r.S_eff - Lc;
+  r.bad = ctx < 1 || ctx > g.max_ctx || Lc < 0 || Lc > g.P * kPage || (Lc > 0 && ctx < g.S + Lc) || r.recent < 0 ||
+          r.recent > g.R;
+  int chunk = (Lc + ns - 1) / ns;
+  chunk = (chunk + 31) & ~31;
+  r.n0 = r.bad ? 0 : min(Lc, j * chunk);
+  r.n1 = r.bad ? 0 : min(Lc, r.n0 + chunk);
+  return r;
+}
+
+__device__ inline void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(src), "r"(bytes) : "memory");
+}
+
 // Programmatic dependent launch: wait until the preceding kernel of the stream
 // has completed and its writes are visible; let the next kernel launch early.
 // Without a programmatic predecessor or successor both are no-ops.
@@ -516,26 +539,34 @@ __global__ void __launch_bounds__(kThr, 1) decode_kernel(
   __syncthreads();
   // The step-t key slice depends on nothing another kernel of a decode sequence writes, so it is
   // fetched before waiting for the preceding kernel in the stream (programmatic dependent launch):
-  // its latency overlaps that kernel's tail.  Everything else is read after the wait.
+  // its latency overlaps that kernel's tail.  Everything else is read after the wait.  Before it,
+  // the counters are read only as a hint (the preceding kernel may still rewrite them; read
+  // through L2, not kept in L1): the split's first key pages and RoPE rows they name are prefetched
+  // into L2, always inside the request's own stream and the RoPE table, so the real copies issued
+  // after the wait find them there.
   if (producer && lane == 0) {
     const uint32_t bk = smem_addr(&bars[0]);
     mbar_expect_tx(bk, X::KS);
     bulk_g2s(smem_addr(Ks), cbp + cbp_slice_off(g, layer, 0, blk, h, s), X::KS, bk);
+    if (!pool) {
+      const SplitRange hint = split_range(g, __ldcg(ctx_len + b), __ldcg(coded_len + b), j, ns);
+      if (hint.n0 < hint.n1) {
+        const int t1 = min(hint.n1, hint.n0 + kStages * kChunk);
+        prefetch_l2_bulk(idx + idx_stream_off(g, layer, blk, b, h, 0) + (size_t)(hint.n0 / kPage) * X::PAGE,
+                         (uint32_t)((t1 - hint.n0 + kPage - 1) / kPage) * X::PAGE);
+        const int r0 = (g.S + hint.n0) >> 3, r1 = (g.S + min(hint.n1, hint.n0 + kChunk) - 1) >> 3;
+        prefetch_l2_bulk(rope + (size_t)r0 * F * 2, (uint32_t)(r1 - r0 + 1) * F * 8);
+      }
+    }
   }
   grid_dependency_wait();
   launch_dependents();
 
   const int ctx = ctx_len[b], Lc = coded_len[b];
-  const int S_eff = min(g.S, max(ctx, 0));
-  const int recent = ctx - S_eff - Lc;
-  const bool bad = ctx < 1 || ctx > g.max_ctx || Lc < 0 || Lc > g.P * kPage ||
-                   (Lc > 0 && ctx < g.S + Lc) || recent < 0 || recent > g.R;
+  const SplitRange sr = split_range(g, ctx, Lc, j, ns);
+  const bool bad = sr.bad;
+  const int S_eff = sr.S_eff, recent = sr.recent, n0 = sr.n0, n1 = sr.n1;
   if (bad && j == 0 && tid == 0) set_status(st, LVQ_ECAPACITY);
-
-  int chunk = (Lc + ns - 1) / ns;
-  chunk = (chunk + 31) & ~31;
-  const int n0 = bad ? 0 : min(Lc, j * chunk);
-  const int n1 = bad ? 0 : min(Lc, n0 + chunk);
   const bool do_coded = n0 < n1;
   const int n_kchunks = do_coded ? (n1 - n0 + kChunk - 1) / kChunk : 0;
   const int n_stream = 2 * n_kchunks;            // per super-chunk: its K chunks, then its V chunks
