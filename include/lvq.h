@@ -175,6 +175,16 @@ LVQ_API const char* lvq_status_string(lvq_status s);
  * LVQ_EINVAL for unknown bits.  lvq_debug_faults(0, 0) restores normal operation. */
 LVQ_API lvq_status lvq_debug_faults(int64_t wait_iters, int32_t fault_mask);
 
+/* Caps the CTAs (one per SM) of the later lvq_decode_attention calls of this process: 0 (the
+ * default) launches one CTA per work item (request, query head, split); max_ctas > 0 launches
+ * at most that many, each walking a contiguous run of work items ordered by KV head, cost-
+ * balanced by coded tokens (the step slices of a KV head are copied once per run, and the next
+ * item's code pages stream in while the current item finishes).  Use it to leave SMs to a
+ * concurrent kernel.  Both grids compute the same attention (the bf16 share's fp32 summation
+ * order differs); on the Ouro-shaped workloads the uncapped grid is as fast or faster.
+ * Process-global, not thread-safe.  LVQ_EINVAL if max_ctas < 0. */
+LVQ_API lvq_status lvq_decode_max_ctas(int32_t max_ctas);
+
 /* Helper: packs the logical codebooks (cb, see lvq_layout.cb_*) into the
  * step-major layout the decoder reads (cbp) and computes each entry's squared
  * norm in fp64, rounded to fp32 (cb_norm, may be NULL).  All device

@@ -40,6 +40,8 @@ lvq_status check_cfg(const lvq_config* c, bool need_table = true) {
 // test hook state (lvq_debug_faults); the defaults leave every kernel as in normal use
 static long debug_wait_iters = kWaitIters;
 static int debug_fault = 0;
+// lvq_decode_max_ctas (0: one decode CTA per work item)
+static int decode_max_ctas = 0;
 
 Geo make_geo(const lvq_config* c) {
   Geo g;
@@ -53,6 +55,7 @@ Geo make_geo(const lvq_config* c) {
   g.page_bytes = g.ng * kPage;
   g.wait_iters = debug_wait_iters;
   g.fault = debug_fault;
+  g.max_ctas = decode_max_ctas;
   g.pool = c->pool_pages;
   g.pts = (g.P + 3) / 4 * 4;       // page-table row: whole 16-byte pieces
   g.pt = c->page_table;
@@ -283,6 +286,12 @@ lvq_status lvq_debug_faults(int64_t wait_iters, int32_t fault_mask) {
   if (fault_mask & ~(kFaultDecodeDropChunk | kFaultKmeansDropTile)) return LVQ_EINVAL;
   debug_wait_iters = wait_iters > 0 ? (long)wait_iters : kWaitIters;
   debug_fault = fault_mask;
+  return LVQ_OK;
+}
+
+lvq_status lvq_decode_max_ctas(int32_t max_ctas) {
+  if (max_ctas < 0) return LVQ_EINVAL;
+  decode_max_ctas = max_ctas;
   return LVQ_OK;
 }
 

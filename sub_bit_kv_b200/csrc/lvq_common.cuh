@@ -24,6 +24,7 @@ struct Geo {
   int pool;          // pool mode: physical pages per (layer, block, head, K/V); 0: per-request streams
   int pts;           // page-table entries per request (pool mode)
   const int32_t* pt; // device page table [B][pts] (pool mode)
+  int max_ctas;      // decode: CTA cap (lvq_decode_max_ctas; 0: one CTA per work item)
 };
 // Test hook bits (lvq_debug_faults): a copy that is never issued, so that a bounded wait
 // runs out and the kernel reports LVQ_ETIMEOUT.

@@ -63,6 +63,7 @@ _SIGS = {
                           ctypes.c_int64, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P],
     "lvq_status_string": [_I32],
     "lvq_debug_faults": [ctypes.c_int64, _I32],
+    "lvq_decode_max_ctas": [_I32],
     "lvq_decode_attention_noalloc": [ctypes.POINTER(lvq_config), ctypes.POINTER(lvq_layout), _I32, _I32, _I32,
                                      _P, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P, _P],
     "lvq_pool_create": [_I32, ctypes.POINTER(_P)],
@@ -220,6 +221,12 @@ def lvq_debug_faults(wait_iters: int = 0, fault_mask: int = 0):
     """Test hook: bound of every device-side wait (0: the normal bound) and copies that never
     happen (bit 0: decode's first code chunk, bit 1: k-means' first tile).  Process-global."""
     _check(lib().lvq_debug_faults(int(wait_iters), int(fault_mask)), "lvq_debug_faults")
+
+
+def lvq_decode_max_ctas(max_ctas: int = 0):
+    """Caps the CTAs of later lvq_decode_attention calls (0: one per work item); with more work
+    items than the cap each CTA walks a run of them.  Process-global."""
+    _check(lib().lvq_decode_max_ctas(int(max_ctas)), "lvq_decode_max_ctas")
 
 
 def lvq_encode_page(cfg, lay, batch, ctx_len, coded_len, ring, cb, cb_norm, idx, dev_status, stream=None):

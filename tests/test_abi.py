@@ -141,6 +141,14 @@ def test_debug_fault_hook_host_side():
     lvq.lvq_debug_faults(0, 0)
 
 
+def test_decode_max_ctas_host_side():
+    with pytest.raises(lvq.LvqError) as e:
+        lvq.lvq_decode_max_ctas(-1)
+    assert e.value.status == lvq.LVQ_EINVAL
+    lvq.lvq_decode_max_ctas(3)
+    lvq.lvq_decode_max_ctas(0)
+
+
 def test_encode_prefill_layer_argument_on_the_host():
     """layer = -1 (every layer in one call) passes the host checks -- on a machine without a
     GPU it then stops at the device check -- while anything below -1 or past the last layer
