@@ -78,6 +78,8 @@ def parse(argv=None):
     ap.add_argument("--pool", action="store_true",
                     help="decode workloads: codes in a shared page pool behind an 8-token page table")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--oracle-procs", type=int, default=0,
+                    help="host processes timing the oracle (0: every usable core, at most %d)" % ORACLE_MAX_PROCS)
     ap.add_argument("--ref-sample", type=int, default=2,
                     help="units (head-attentions, or encode batches) per step of the reference (oracle) arm")
     ap.add_argument("--profile", default="", choices=["", "decode", "encode", "kmeans"],
@@ -88,18 +90,37 @@ def parse(argv=None):
     return args
 
 
-# DRAM bytes (read + write) of one decode_kernel<128,4> launch of the headline workload, from
-# one ncu capture (`python bench.py --profile decode` under ncu), valid only for the decode
-# source it was taken on: the bench reports it when the file's hash still matches, else null.
-DECODE_TRAFFIC = {"source_sha256": "e9422eb0c0c52da9d84373c6bdacf44bd53c0350259b6b29ed0d4d54ef5ada21",
-                  "bytes_per_launch": 36771200}
+# One ncu capture of a decode_kernel<128,4> launch of the headline workload
+# (`python bench.py --profile decode` under ncu): its DRAM bytes (read + write) and its warp
+# instructions (smsp__inst_executed.sum), valid only for the decode source they were taken on:
+# the bench reports them when the file's hash still matches, else null.
+DECODE_NCU = {"source_sha256": "6697790a9e2006d98c668dd7242a1d35d8756438b863a515f91c8f4ced17088d",
+              "dram_bytes_per_launch": 36983296, "warp_inst_per_launch": 15338781}
 
 
-def decode_traffic():
+def _decode_ncu():
     src = os.path.join(ROOT, "sub_bit_kv_b200", "csrc", "lvq_decode.cu")
     with open(src, "rb") as f:
         sha = hashlib.sha256(f.read()).hexdigest()
-    return DECODE_TRAFFIC["bytes_per_launch"] if sha == DECODE_TRAFFIC["source_sha256"] else None
+    return DECODE_NCU if sha == DECODE_NCU["source_sha256"] else None
+
+
+def decode_traffic():
+    n = _decode_ncu()
+    return n["dram_bytes_per_launch"] if n else None
+
+
+def decode_issue(launch_ms, sm_mhz, n_sm, token_heads):
+    """The issue ceiling of one decode launch: its warp instructions (ncu) issued at one per
+    scheduler per cycle (4 per SM) at the SM clock sampled during the timed region; `frac` is
+    that ceiling's duration over the measured one."""
+    n = _decode_ncu()
+    if not n or not sm_mhz:
+        return None
+    inst = n["warp_inst_per_launch"]
+    ceiling_ms = inst / (n_sm * 4 * sm_mhz * 1e6) * 1e3
+    return {"warp_inst_per_launch": inst, "per_coded_token_head": inst / token_heads, "sm_mhz": sm_mhz,
+            "ceiling_us": ceiling_ms * 1e3, "frac": ceiling_ms / launch_ms}
 
 
 def _peaks_file():
@@ -229,6 +250,21 @@ def encode_config(w, world: int) -> dict:
 
 # ------------------------------------------------------------------------------ oracle baselines
 
+ORACLE_MAX_PROCS = 32      # host processes of the oracle baselines (each one thread)
+
+
+def oracle_procs(requested: int = 0) -> int:
+    """Host processes for the oracle: `requested`, else every core this process may use, at most
+    ORACLE_MAX_PROCS (each holds its own copy of the inputs)."""
+    if requested > 0:
+        return requested
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        n = os.cpu_count() or 1
+    return max(1, min(n, ORACLE_MAX_PROCS))
+
+
 def _one_thread():
     try:
         from threadpoolctl import threadpool_limits
@@ -335,71 +371,103 @@ class _OracleEncode:
         return el
 
 
-def cpu_baseline(name: str, seconds: float):
-    """The oracle on a bounded sample of workload `name` (one host core)."""
-    limiter = _one_thread()
-    try:
-        if name == ENCODE_WORKLOAD:
-            oe = _OracleEncode()
-            n, el = 0, 0.0
-            while el < seconds:
-                el += oe.run(1)
-                n += oe.BATCH
-            return {"value": n / el, "unit": "vectors/s", "cores": 1, "kind": "oracle",
-                    "sample": f"{n} joint vectors of one layer, brute-force nearest of 256 entries (fp64 numpy, "
-                              f"1 thread), per vector; the workload has 48 layers x 33.5 M vectors"}
-        od = _OracleDecode(name)
+def _oracle_proc(name, seconds, count, warm, offset, barrier, queue):
+    """One host process of an oracle baseline (spawned, one thread): builds the workload's oracle
+    inputs, runs `warm` untimed units, waits for every process at `barrier`, then runs units until
+    `seconds` of oracle time have passed (or `count` units); puts (units, oracle seconds, rate in
+    the workload's unit, description) on `queue`."""
+    for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ[var] = "1"
+    _one_thread()
+    if name == ENCODE_WORKLOAD:
+        o = _OracleEncode()
+        o.i = offset
+        o.run(max(warm, 1))
+        barrier.wait(timeout=900)
         n, el = 0, 0.0
-        while el < seconds:
-            el += od.run(1)
+        while (n < count) if count else (el < seconds):
+            el += o.run(1)
             n += 1
-        nu = 8 if od.w.gen_tokens else 0
-        ue = od.page_units(nu) if nu else 0.0
-        value = od.tokens_per_s(el, n, ue, nu)
-        extra = f" plus {nu} page-encode units ({od.units_per_token:.0f} per token)" if nu else ""
-        return {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                "sample": f"{n} single-head decode attentions (requests in turn, contexts "
-                          f"{min(od.ctx)}-{max(od.ctx)}){extra} (fp64 numpy, 1 thread), scaled by "
-                          f"{od.per_token} head-attentions per generated token"}
+        queue.put((n * o.BATCH, el, n * o.BATCH / el, ""))
+        return
+    o = _OracleDecode(name)
+    for b in range(len(o.ctx)):
+        o._codes(b)                                    # every request's inputs exist before the clock
+    o.n = offset
+    o.run(max(warm, 1))
+    barrier.wait(timeout=900)
+    n, el = 0, 0.0
+    while (n < count) if count else (el < seconds):
+        el += o.run(1)
+        n += 1
+    nu = 8 if o.w.gen_tokens else 0
+    ue = o.page_units(nu) if nu else 0.0
+    extra = f" plus {nu} page-encode units ({o.units_per_token:.0f} per token)" if nu else ""
+    queue.put((n, el + ue, o.tokens_per_s(el, n, ue, nu),
+               f"(requests in turn, contexts {min(o.ctx)}-{max(o.ctx)}){extra}, scaled by {o.per_token} "
+               f"head-attentions per generated token"))
+
+
+def oracle_parallel(name: str, procs: int, seconds: float = 0.0, count: int = 0, warm: int = 0):
+    """The oracle on `procs` host processes at once (spawned, one thread each, each sampling other
+    heads and requests); returns the per-process results of _oracle_proc."""
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    barrier, queue = ctx.Barrier(procs), ctx.Queue()
+    ps = [ctx.Process(target=_oracle_proc, args=(name, seconds, count, warm, 7 * i, barrier, queue))
+          for i in range(procs)]
+    for p in ps:
+        p.start()
+    try:
+        res = [queue.get(timeout=1800) for _ in ps]
     finally:
-        if limiter is not None:
-            limiter.unregister()
+        for p in ps:
+            p.join(timeout=60)
+    return res
+
+
+def cpu_baseline(name: str, seconds: float, procs: int = 0):
+    """The oracle on a bounded sample of workload `name`: one single-threaded process per usable
+    host core (at most ORACLE_MAX_PROCS), all timed at once; the rate is their sum."""
+    P = oracle_procs(procs)
+    res = oracle_parallel(name, P, seconds=seconds)
+    value = sum(r[2] for r in res)
+    units = sum(r[0] for r in res)
+    if name == ENCODE_WORKLOAD:
+        return {"value": value, "unit": "vectors/s", "cores": P, "kind": "oracle",
+                "sample": f"{units} joint vectors of one layer over {P} processes (~{seconds:.0f} s each), "
+                          f"brute-force nearest of 256 entries (fp64 numpy, 1 thread per process), per vector; "
+                          f"the workload has 48 layers x 33.5 M vectors"}
+    return {"value": value, "unit": "tokens/s", "cores": P, "kind": "oracle",
+            "sample": f"{units} single-head decode attentions over {P} processes (~{seconds:.0f} s each) "
+                      f"{res[0][3]} (fp64 numpy, 1 thread per process)"}
 
 
 def reference_arm(args):
-    """The oracle on the host: W untimed steps, then K timed steps, each step a bounded sample
-    of the workload (args.ref_sample head-attentions, or encode batches of 1024 vectors),
-    scaled to the metric's unit."""
+    """The oracle on the host: one single-threaded process per usable core (at most
+    ORACLE_MAX_PROCS), each running W untimed steps then K timed steps of a bounded sample of the
+    workload (args.ref_sample head-attentions, or encode batches of 1024 vectors); the rate, in the
+    metric's unit, is the processes' sum."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    limiter = _one_thread()
-    try:
-        if args.workload == ENCODE_WORKLOAD:
-            oe = _OracleEncode()
-            for _ in range(args.warmup):
-                oe.run(args.ref_sample)
-            el = sum(oe.run(args.ref_sample) for _ in range(args.steps))
-            value, unit = args.steps * args.ref_sample * oe.BATCH / el, "vectors/s"
-            sample = (f"{args.steps} steps of {args.ref_sample} batches of {oe.BATCH} joint vectors of one layer, "
-                      f"brute-force nearest entry (fp64 numpy, 1 thread), per vector")
-            config = encode_config(oe.w, args.gpus)
-        else:
-            od = _OracleDecode(args.workload)
-            for _ in range(args.warmup):
-                od.run(args.ref_sample)
-            el = sum(od.run(args.ref_sample) for _ in range(args.steps))
-            nu = 8 if od.w.gen_tokens else 0
-            ue = od.page_units(nu) if nu else 0.0
-            value, unit = od.tokens_per_s(el, args.steps * args.ref_sample, ue, nu), "tokens/s"
-            sample = (f"{args.steps} steps of {args.ref_sample} single-head decode attentions (fp64 numpy, 1 thread), "
-                      f"scaled by {od.per_token} head-attentions per generated token")
-            el += ue
-            config = decode_config(od.w, args.gpus, choose_splits(od.w, 148))
-    finally:
-        if limiter is not None:
-            limiter.unregister()
-    cb = {"value": value, "unit": unit, "cores": 1, "kind": "oracle", "sample": sample}
+    from sub_bit_kv_b200 import synth
+    P = oracle_procs(args.oracle_procs)
+    res = oracle_parallel(args.workload, P, count=args.steps * args.ref_sample, warm=args.warmup * args.ref_sample)
+    value = sum(r[2] for r in res)
+    el = max(r[1] for r in res)                 # host seconds of the slowest process over the K steps
+    if args.workload == ENCODE_WORKLOAD:
+        unit = "vectors/s"
+        sample = (f"{P} processes x {args.steps} steps of {args.ref_sample} batches of {_OracleEncode.BATCH} joint "
+                  f"vectors of one layer, brute-force nearest entry (fp64 numpy, 1 thread per process), per vector")
+        config = encode_config(synth.WORKLOADS[ENCODE_WORKLOAD], args.gpus)
+    else:
+        w = synth.WORKLOADS[args.workload]
+        unit = "tokens/s"
+        sample = (f"{P} processes x {args.steps} steps of {args.ref_sample} single-head decode attentions "
+                  f"{res[0][3]} (fp64 numpy, 1 thread per process)")
+        config = decode_config(w, args.gpus, choose_splits(w, 148))
+    cb = {"value": value, "unit": unit, "cores": P, "kind": "oracle", "sample": sample}
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             # the host time of one sampled step (the rate above is scaled to the workload's unit)
@@ -815,7 +883,7 @@ def decode_arm(args, torch, dist, lvq, synth, world, rank, local, device):
 
     if rank != 0:
         return None
-    cb = cpu_baseline(args.workload, args.cpu_seconds)
+    cb = cpu_baseline(args.workload, args.cpu_seconds, args.oracle_procs)
     clocks = clk.summary()
     return {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -828,6 +896,8 @@ def decode_arm(args, torch, dist, lvq, synth, world, rank, local, device):
                      "traffic": decode_traffic() if args.workload == WORKLOAD else None,
                      "kernel": f"decode_kernel<{d},{lay.c}>",
                      "peak_kind": peak_kind, "bytes_per_launch": bpl, "launch_ms": per_call_ms},
+        "issue": (decode_issue(per_call_ms, clocks.get("sm_mhz"), torch.cuda.get_device_properties(device).multi_processor_count,
+                               sum(coded_now) * w.n_q_heads) if args.workload == WORKLOAD else None),
         "code_stream_GBps": code_stream,
         "page_encode_us": page_us,
         "cpu_baseline": cb,
@@ -922,7 +992,7 @@ def encode_arm(args, torch, dist, lvq, synth, world, rank, local, device):
 
     if rank != 0:
         return None
-    cb = cpu_baseline(ENCODE_WORKLOAD, args.cpu_seconds)
+    cb = cpu_baseline(ENCODE_WORKLOAD, args.cpu_seconds, args.oracle_procs)
     return {
         "metric": METRIC, "value": value, "unit": "vectors/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": per_call_ms, "higher_is_better": True, "scaling": "weak",

@@ -60,3 +60,16 @@ def test_choose_splits():
     assert bench.choose_splits(ws["ouro14_g32_b32"], 148) == 3         # 512 heads: ~6K-token splits
     tiny = dataclasses.replace(ws["tiny"], batch=1)
     assert bench.choose_splits(tiny, 148) == 128                        # capped
+
+
+def test_decode_issue_ceiling(monkeypatch):
+    """Warp instructions issued at one per scheduler per cycle, 4 schedulers per SM: 148 SMs at
+    1000 MHz issue 5.92e11 per second, so 5.92e6 instructions take 10 us."""
+    monkeypatch.setattr(bench, "_decode_ncu", lambda: {"warp_inst_per_launch": 5.92e6})
+    got = bench.decode_issue(launch_ms=0.020, sm_mhz=1000, n_sm=148, token_heads=1000)
+    assert abs(got["ceiling_us"] - 10.0) < 1e-9
+    assert abs(got["frac"] - 0.5) < 1e-12
+    assert got["per_coded_token_head"] == 5.92e3
+    assert bench.decode_issue(0.02, None, 148, 1000) is None            # no clock sample
+    monkeypatch.setattr(bench, "_decode_ncu", lambda: None)              # another decode source
+    assert bench.decode_issue(0.02, 1000, 148, 1000) is None
