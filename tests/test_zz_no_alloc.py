@@ -73,6 +73,30 @@ def test_noalloc_clears_the_counters_of_each_layout():
         assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
 
 
+def test_noalloc_after_a_timed_out_call():
+    """A noalloc call whose bounded waits run out (test hook: a copy that never happens) reports
+    LVQ_ETIMEOUT and leaves the shared array's counters exact: the next noalloc call matches the
+    workspace path bit for bit."""
+    w = dataclasses.replace(synth.WORKLOADS["ouro14_g16_32k"], n_layers=1, n_kv_heads=2, n_q_heads=2)
+    case = Hl.build_case(w, layers=1, ctx=[1500], max_splits=8)
+    c = case.cache
+    q = synth.queries(w, 0, 3, batch=1).cuda()
+    out = torch.empty(1, w.n_q_heads, w.head_dim, dtype=torch.float32, device="cuda")
+    lse = torch.empty(1, w.n_q_heads, dtype=torch.float32, device="cuda")
+    lvq.lvq_debug_faults(1 << 12, 1)
+    try:
+        lvq.lvq_decode_attention_noalloc(case.cfg, c.lay, 0, 3, 1, q, c.ctx_len, c.coded_len, c.sink, c.ring, c.idx,
+                                         c.cbp, c.rope, 4, out, lse, c.status)
+        torch.cuda.synchronize()
+    finally:
+        lvq.lvq_debug_faults(0, 0)
+    assert int(c.status.item()) == lvq.LVQ_ETIMEOUT
+    c.status.zero_()
+    got_out, got_lse = _call(case, lvq.lvq_decode_attention_noalloc, 0, 3, q, 4)
+    ref_out, ref_lse = _call(case, lvq.lvq_decode_attention, 0, 3, q, 4, ws=(c.workspace,))
+    assert torch.equal(got_out, ref_out) and torch.equal(got_lse, ref_lse)
+
+
 def test_noalloc_rejects_a_layout_beyond_its_array():
     """Checked on the host before anything is launched."""
     w = dataclasses.replace(synth.WORKLOADS["ouro14_g16_32k"], n_layers=1)
