@@ -13,8 +13,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 @pytest.mark.parametrize("workload,unit", [("ouro14_g16_32k", "tokens/s"), ("ouro26_prefill_32k", "vectors/s")])
 def test_reference_arm_line_has_the_contract_keys(workload, unit):
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
-                        "--warmup", "0", "--ref-sample", "1", "--workload", workload], capture_output=True,
-                       text=True, timeout=600, cwd=ROOT)
+                        "--warmup", "0", "--ref-sample", "1", "--oracle-procs", "2", "--workload", workload],
+                       capture_output=True, text=True, timeout=600, cwd=ROOT)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
     assert len(lines) == 1
@@ -25,5 +25,13 @@ def test_reference_arm_line_has_the_contract_keys(workload, unit):
     assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
     assert d["config"]["workload"] == workload and d["unit"] == unit
     cb = d["cpu_baseline"]
-    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert cb["kind"] == "oracle" and cb["cores"] == 2 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"]["value"] == d["value"] and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_oracle_processes_default_to_the_usable_cores():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.oracle_procs(3) == 3
+    n = bench.oracle_procs()
+    assert 1 <= n <= bench.ORACLE_MAX_PROCS and n <= len(os.sched_getaffinity(0))
