@@ -372,3 +372,34 @@ def test_decode_large_score_range():
     for step in range(w.T):
         q = synth.queries(w, 0, step).cuda()
         _check_decode(case, 0, step, q, 1)
+
+
+@pytest.mark.parametrize("cap", [0, 2])
+def test_decode_reports_counters_outside_the_layout(cap):
+    """A request whose counters the layout cannot hold (its recent window longer than the ring)
+    is reported as LVQ_ECAPACITY and left empty (output 0, lse -inf); the other requests of
+    the launch are computed as usual.  cap = 2: two CTAs walking runs of items."""
+    w = _reduced("ouro14_g16_32k", n_layers=1, n_kv_heads=2, n_q_heads=2)
+    ctx = [4 + 900 + 128, 4 + 500 + 128, 4 + 300 + 128]
+    case = Hl.build_case(w, layers=1, ctx=ctx, max_splits=8)
+    c = case.cache
+    c.coded_len[1] = case.coded[1] - (c.lay.ring_tokens + 5)       # recent window > ring
+    q = synth.queries(w, 0, 1, batch=3).cuda()
+    out = torch.empty(3, w.n_q_heads, w.head_dim, dtype=torch.float32, device="cuda")
+    lse = torch.empty(3, w.n_q_heads, dtype=torch.float32, device="cuda")
+    lvq.lvq_decode_max_ctas(cap)
+    try:
+        lvq.lvq_decode_attention(case.cfg, c.lay, 0, 1, 3, q, c.ctx_len, c.coded_len, c.sink, c.ring, c.idx, c.cbp,
+                                 c.rope, 4, c.workspace, out, lse, c.status)
+        torch.cuda.synchronize()
+    finally:
+        lvq.lvq_decode_max_ctas(0)
+    assert int(c.status.item()) == lvq.LVQ_ECAPACITY
+    out, lse = out.cpu(), lse.cpu()
+    assert torch.equal(out[1], torch.zeros_like(out[1])) and bool(torch.isneginf(lse[1]).all())
+    for b in (0, 2):
+        for hq in range(w.n_q_heads):
+            ro, rl, _ = Hl.oracle_decode(case, 0, 1, b, hq, q)
+            assert float(np.abs(out[b, hq].numpy() - ro).max()) <= Hl.OUT_ATOL
+            Hl.assert_lse_close(float(lse[b, hq]), rl)
+    c.status.zero_()
