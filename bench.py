@@ -75,6 +75,9 @@ def parse(argv=None):
     ap.add_argument("--splits", type=int, default=0, help="split count (0: choose)")
     ap.add_argument("--workload", default=WORKLOAD, choices=list(DECODE_WORKLOADS) + [ENCODE_WORKLOAD])
     ap.add_argument("--no-encode", action="store_true", help="skip the one-layer prefill-encode measurement")
+    ap.add_argument("--max-ctas", type=int, default=0,
+                    help="decode workloads: cap the decode's CTAs (lvq_decode_max_ctas); below the work-item "
+                         "count each CTA walks a run of items")
     ap.add_argument("--pool", action="store_true",
                     help="decode workloads: codes in a shared page pool behind an 8-token page table")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -751,6 +754,8 @@ def _setup(args):
     if world > 1:
         dist.barrier()
     lvq.lib()
+    if getattr(args, "max_ctas", 0):
+        lvq.lvq_decode_max_ctas(args.max_ctas)
     return torch, dist, lvq, synth, world, rank, local, device
 
 
@@ -885,19 +890,26 @@ def decode_arm(args, torch, dist, lvq, synth, world, rank, local, device):
         return None
     cb = cpu_baseline(args.workload, args.cpu_seconds, args.oracle_procs)
     clocks = clk.summary()
+    # the launch's kernel: with a CTA cap below the work items, CTAs walk runs of items
+    runs = bool(args.max_ctas) and B * Hq * ns > min(args.max_ctas, n_sm)
+    headline_kernel = args.workload == WORKLOAD and not runs      # the kernel the ncu counters describe
+    extra_cfg = {}
+    if args.pool:
+        extra_cfg["codes"] = f"page pool, {POOL_BITE}-page bites"
+    if args.max_ctas:
+        extra_cfg["max_ctas"] = args.max_ctas
     return {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": dict(decode_config(w, world, ns), **({"codes": f"page pool, {POOL_BITE}-page bites"} if args.pool
-                                                         else {})),
+        "config": dict(decode_config(w, world, ns), **extra_cfg),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak,
-                     "traffic": decode_traffic() if args.workload == WORKLOAD else None,
-                     "kernel": f"decode_kernel<{d},{lay.c}>",
+                     "traffic": decode_traffic() if headline_kernel else None,
+                     "kernel": f"decode_runs_kernel<{d},{lay.c}>" if runs else f"decode_kernel<{d},{lay.c}>",
                      "peak_kind": peak_kind, "bytes_per_launch": bpl, "launch_ms": per_call_ms},
-        "issue": (decode_issue(per_call_ms, clocks.get("sm_mhz"), torch.cuda.get_device_properties(device).multi_processor_count,
-                               sum(coded_now) * w.n_q_heads) if args.workload == WORKLOAD else None),
+        "issue": (decode_issue(per_call_ms, clocks.get("sm_mhz"), n_sm, sum(coded_now) * w.n_q_heads)
+                  if headline_kernel else None),
         "code_stream_GBps": code_stream,
         "page_encode_us": page_us,
         "cpu_baseline": cb,
