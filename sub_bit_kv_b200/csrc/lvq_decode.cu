@@ -1357,7 +1357,6 @@ __global__ void __launch_bounds__(kThr, 1) decode_runs_kernel(
   const bool producer = warp == kCW;
   const int gq = g.Hq / g.H;
   const int blk = step / g.Tc, s = step % g.Tc;
-  const int n_items = g.H * batch * ns * gq;
   int32_t* counters = reinterpret_cast<int32_t*>(ws + (size_t)g.B * g.Hq * g.max_splits * 2 * (D + 2));
   auto slot_of = [&](const Item& x) { return ((size_t)x.b * g.Hq + x.hq) * g.max_splits * 2; };
 
@@ -1508,8 +1507,9 @@ __global__ void __launch_bounds__(kThr, 1) decode_runs_kernel(
         }
       };
       bool to = aborted();
-      // (1) the previous item's slices released (the next value slice overwrites its value slice, a
-      // new KV head its key slice); the ring keeps being fed meanwhile
+      // (1) the previous item is done with the step slices (a new KV head overwrites them); every
+      // item's release is awaited, in order, so that the barrier's phases stay paired.  The ring
+      // keeps being fed meanwhile.
       if (k > 0 && !to) {
         bool done = false;
         for (long i = 0; i < wit && !done; ++i) {
