@@ -97,7 +97,7 @@ def parse(argv=None):
 # (`python bench.py --profile decode` under ncu): its DRAM bytes (read + write) and its warp
 # instructions (smsp__inst_executed.sum), valid only for the decode source they were taken on:
 # the bench reports them when the file's hash still matches, else null.
-DECODE_NCU = {"source_sha256": "d80dc3c957a0b25469991add426ed361e81cd8d56f93e340d86b1f1cf1f0d000",
+DECODE_NCU = {"source_sha256": "3d24c45237a893e6b9f0d88fdb2b00c9fd52fe726cf3de34b51dd97015c8fed9",
               "dram_bytes_per_launch": 36983296, "warp_inst_per_launch": 15338781}
 
 
